@@ -1,0 +1,102 @@
+"""Seeded synthetic inputs for the attention forward pass.
+
+This module is shared by the tests, the smoke check and the benchmark, and it
+is the only thing the CUDA path's callers and the oracle's callers share.  It
+holds no attention arithmetic: it only names the workloads and draws q, k, v.
+
+Recipe: torch.Generator('cpu').manual_seed(seed); q, k, v are drawn in that
+order as float32 standard normals of the layout's shape, multiplied by the
+workload's standard deviation, and rounded to nearest into fp16 / bf16.  The
+seed 42 is the one the accuracy check on the pages uses (page "ops-transformer
+FlashAttention on Atlas 800", section "accuracy check"); workload n uses 42 + n.
+"""
+import math
+from dataclasses import dataclass, replace
+
+import torch
+
+DTYPES = {"fp16": torch.float16, "bf16": torch.bfloat16}
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    dtype: str          # "fp16" | "bf16"
+    layout: str         # "BSND" ([B, S, H, D]) | "BHSD" ([B, H, S, D])
+    B: int
+    H: int
+    Sq: int
+    Sk: int
+    D: int
+    causal: bool
+    scale: float
+    qk_std: float = 1.0
+    v_std: float = 1.0
+    seed: int = 42
+
+    def q_shape(self):
+        return (self.B, self.Sq, self.H, self.D) if self.layout == "BSND" else (self.B, self.H, self.Sq, self.D)
+
+    def kv_shape(self):
+        return (self.B, self.Sk, self.H, self.D) if self.layout == "BSND" else (self.B, self.H, self.Sk, self.D)
+
+    def flops(self):
+        """Attention-forward flops 4*B*H*Sq*Sk*D, halved when causal (the metric's convention)."""
+        f = 4.0 * self.B * self.H * self.Sq * self.Sk * self.D
+        return f / 2 if self.causal else f
+
+    def with_(self, **kw):
+        return replace(self, **kw)
+
+
+# The five workloads the measurements are quoted on.
+WORKLOADS = {
+    "fp16_bsnd_b1_h2_s512_d64": Workload(
+        "fp16_bsnd_b1_h2_s512_d64", "fp16", "BSND", 1, 2, 512, 512, 64, False, 1.0 / 8, seed=42),
+    "fp16_bhsd_b8_h32_s4096_d128_causal": Workload(
+        "fp16_bhsd_b8_h32_s4096_d128_causal", "fp16", "BHSD", 8, 32, 4096, 4096, 128, True,
+        1.0 / math.sqrt(128), seed=43),
+    "bf16_bhsd_b2_h40_s8192_d128_causal": Workload(
+        "bf16_bhsd_b2_h40_s8192_d128_causal", "bf16", "BHSD", 2, 40, 8192, 8192, 128, True,
+        1.0 / math.sqrt(128), seed=44),
+    "bf16_bhsd_b1_h8_s65536_d128_causal": Workload(
+        "bf16_bhsd_b1_h8_s65536_d128_causal", "bf16", "BHSD", 1, 8, 65536, 65536, 128, True,
+        1.0 / math.sqrt(128), seed=45),
+    "bf16_bsnd_b1_h32_s16000_d128_qk3": Workload(
+        "bf16_bsnd_b1_h32_s16000_d128_qk3", "bf16", "BSND", 1, 32, 16000, 16000, 128, False,
+        1.0 / math.sqrt(128), qk_std=3.0, seed=46),
+}
+WORKLOAD_ORDER = list(WORKLOADS)
+BENCH_WORKLOAD = "bf16_bhsd_b2_h40_s8192_d128_causal"
+
+
+def make_qkv(w: Workload, device="cpu"):
+    """Draws q, k, v for workload w (see the module docstring for the recipe)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(w.seed))
+    dt = DTYPES[w.dtype]
+    q = (torch.randn(w.q_shape(), generator=g, dtype=torch.float32) * w.qk_std).to(dt)
+    k = (torch.randn(w.kv_shape(), generator=g, dtype=torch.float32) * w.qk_std).to(dt)
+    v = (torch.randn(w.kv_shape(), generator=g, dtype=torch.float32) * w.v_std).to(dt)
+    if device != "cpu":
+        q, k, v = q.to(device), k.to(device), v.to(device)
+    return q, k, v
+
+
+def sample_rows(w: Workload, per_head_first=64, per_head_last=64, stride=97, max_rows=None):
+    """Flat row ids (b * H + h) * Sq + i for a stratified sample of every head.
+
+    Each head contributes its first rows, every stride-th row and its last rows,
+    so that the first and last query tiles, the diagonal and the ragged tail
+    are all represented.
+    """
+    rows = []
+    for bh in range(w.B * w.H):
+        picked = set(range(min(per_head_first, w.Sq)))
+        picked.update(range(0, w.Sq, stride))
+        picked.update(range(max(0, w.Sq - per_head_last), w.Sq))
+        rows.extend(bh * w.Sq + i for i in sorted(picked))
+    if max_rows is not None and len(rows) > max_rows:
+        step = len(rows) / max_rows
+        rows = [rows[int(j * step)] for j in range(max_rows)]
+    return rows
