@@ -1,0 +1,198 @@
+"""B200 (sm_100a) FlashAttention forward: Python binding of libfa_fwd.so.
+
+The binding only marshals arguments: it reads pointers, shapes and the
+current CUDA stream from torch tensors and calls the C ABI declared in
+include/fa_fwd.h.  Every step of the computation runs in the library's CUDA
+kernel.  There is no CPU fallback: if the library cannot be loaded, importing
+the entry points raises.
+
+    from attention_forward_19_b200 import flash_attention_forward
+    o, lse = flash_attention_forward(q, k, v, layout="BHSD", causal=True)
+
+The C entry points are also exposed under their own names (fa_fwd,
+fa_device_status, fa_query_support, fa_status_string, fa_last_cuda_error,
+fa_version) with the same arguments as in the header.
+"""
+import ctypes
+import math
+import os
+
+from . import build as _build
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_NOT_DEVICE_POINTER = 3
+FA_ERR_MISALIGNED = 4
+FA_ERR_ALIAS = 5
+FA_ERR_CUDA = 6
+FA_ERR_TIMEOUT = 7
+
+FA_BSND = 0
+FA_BHSD = 1
+FA_FP16 = 0
+FA_BF16 = 1
+
+LAYOUTS = {"BSND": FA_BSND, "BHSD": FA_BHSD}
+
+# Names every public symbol of include/fa_fwd.h.
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_device_status", "fa_query_support", "fa_status_string",
+                    "fa_last_cuda_error", "fa_version")
+
+
+class FaError(RuntimeError):
+    """A non-zero fa_status returned by the library."""
+
+    def __init__(self, status, where):
+        self.status = status
+        name = fa_status_string(status) if _LIB is not None else str(status)
+        extra = ""
+        if status == FA_ERR_CUDA and _LIB is not None:
+            extra = f" (CUDA error {fa_last_cuda_error()})"
+        super().__init__(f"{where}: {name}{extra}")
+
+
+_LIB = None
+
+
+def library_path():
+    return _build.LIB
+
+
+def load_library(path=None, rebuild_if_stale=True):
+    """Loads libfa_fwd.so (compiling it first if missing or stale and nvcc is available)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if path is None:
+        path = _build.LIB
+        if rebuild_if_stale and os.path.exists(_build.NVCC):
+            _build.build()
+    if not os.path.exists(path):
+        raise ImportError(f"the CUDA library {path} is missing; run python -m attention_forward_19_b200.build")
+    lib = ctypes.CDLL(path)
+    i64, vp, c_int, c_float = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.fa_fwd.restype = c_int
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, vp]
+    lib.fa_device_status.restype = c_int
+    lib.fa_device_status.argtypes = [vp]
+    lib.fa_query_support.restype = c_int
+    lib.fa_query_support.argtypes = [i64, c_int]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_status_string.argtypes = [c_int]
+    lib.fa_last_cuda_error.restype = c_int
+    lib.fa_last_cuda_error.argtypes = []
+    lib.fa_version.restype = c_int
+    lib.fa_version.argtypes = []
+    _LIB = lib
+    return lib
+
+
+# ----------------------------------------------------------------------------- raw C entry points
+
+
+def fa_fwd(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, stream):
+    """The C fa_fwd with raw pointers (ints) and sizes; returns the fa_status code."""
+    lib = load_library()
+    return lib.fa_fwd(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
+                      int(bool(causal)), float(scale), int(dtype), stream)
+
+
+def fa_device_status(stream=None):
+    return load_library().fa_device_status(stream)
+
+
+def fa_query_support(D, dtype):
+    return load_library().fa_query_support(int(D), int(dtype))
+
+
+def fa_status_string(status):
+    return load_library().fa_status_string(int(status)).decode()
+
+
+def fa_last_cuda_error():
+    return load_library().fa_last_cuda_error()
+
+
+def fa_version():
+    return load_library().fa_version()
+
+
+# ----------------------------------------------------------------------------- torch convenience
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.float16:
+        return FA_FP16
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float16 or bfloat16")
+
+
+def _dims(q, k, layout, head_num=None):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be 4-D")
+    if layout == FA_BSND:
+        B, Sq, H, D = q.shape
+        Bk, Sk, Hk, Dk = k.shape
+    else:
+        B, H, Sq, D = q.shape
+        Bk, Hk, Sk, Dk = k.shape
+    if (Bk, Hk, Dk) != (B, H, D):
+        raise ValueError(f"q {tuple(q.shape)} and k {tuple(k.shape)} do not match in layout "
+                         f"{'BSND' if layout == FA_BSND else 'BHSD'}")
+    if head_num is not None and head_num != H:
+        raise ValueError(f"head_num mismatch: head_num={head_num} but the tensors hold {H} heads")
+    return B, H, Sq, Sk, D
+
+
+def flash_attention_forward(q, k, v, layout="BSND", causal=False, scale=None, head_num=None,
+                            out=None, lse=None, stream=None):
+    """Attention forward on CUDA tensors through the C ABI.
+
+    q: [B, Sq, H, D] (BSND) or [B, H, Sq, D] (BHSD); k, v likewise with Sk.
+    scale=None uses 1/sqrt(D).  Returns (o, lse): o like q, lse fp32 [B, H, Sq].
+    out / lse may be given to reuse buffers.  Runs on `stream` (default: the
+    current torch stream) without synchronising.
+    """
+    import torch
+    lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    B, H, Sq, Sk, D = _dims(q, k, lay, head_num)
+    if v.shape != k.shape:
+        raise ValueError(f"v {tuple(v.shape)} must have k's shape {tuple(k.shape)}")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous in the stated layout")
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v must share one dtype")
+    dt = _dtype_code(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    if out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor like q")
+    if lse.shape != (B, H, Sq) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 tensor of shape [B, H, Sq]")
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device) if q.is_cuda else None
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                B, H, Sq, Sk, D, lay, causal, scale, dt, sptr)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd")
+    return out, lse
+
+
+def check_device_status(stream=None):
+    """Synchronises the stream and raises FaError if a kernel reported a wait timeout."""
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    st = fa_device_status(sptr)
+    if st != FA_OK:
+        raise FaError(st, "fa_device_status")

@@ -1,0 +1,1013 @@
+// fa_fwd.cu -- FlashAttention forward for NVIDIA B200 (sm_100a) and its C ABI.
+//
+// What is computed (the method of the pages, restated):
+//   O = softmax(scale * Q K^T [+ causal mask]) V per (batch, head), and the
+//   natural-log log-sum-exp of every row.  The key axis is walked tile by
+//   tile with an online softmax -- a running row max m and a running exp-sum
+//   l, both rescaled whenever m grows, with the partial output rescaled the
+//   same way -- so the score matrix never leaves the chip.
+//   Page "FlashAttention: long-text inference without running out of memory"
+//   (ai6s.net/6a0d42d8), section "FlashAttention's answer: tiling + online
+//   normalisation" (the m / l recurrence); page "catlass FlashAttention
+//   template tuning" (hwcomputing.csdn.net/6a0d4681), section "causal mask
+//   implementations", mode 2 (skip key tiles above the diagonal, mask inside
+//   diagonal tiles); page "64K long-sequence FlashAttention"
+//   (ai6s.net/6a140d07), section "layer 2: numerical stability" (the per-row
+//   LSE) and section "multi-AI-Core load balancing" (balanced scheduling of
+//   uneven tile counts).
+//
+// How it maps onto sm_100a (a design of its own, not the pages' Ascend one):
+//   * One persistent CTA per SM (10 warps, 320 threads).  A work unit is two
+//     128-row query tiles of one (batch, head); units are walked longest
+//     first inside L2-sized groups of heads (static schedule, no workspace).
+//   * Warp 8 (load): TMA loads of Q tiles and a ring of K / V tiles
+//     (128 keys x D, 128-byte swizzle) behind full / empty mbarriers.
+//   * Warp 9 (MMA): one thread issues tcgen05.mma.  S_t = Q_t K^T goes to
+//     tensor memory (fp32, 128 lanes x 128 columns); O_t += P_t V reads P_t
+//     from tensor memory (it overwrites the first 64 columns of S_t) and V
+//     from shared memory.  TMEM: S0 | S1 | O0 | O1 = 512 columns.
+//   * Warps 0-3 / 4-7 (softmax warpgroups, one per query tile): each thread
+//     owns one query row.  It reads its S row from TMEM, masks it (diagonal
+//     and ragged-tail tiles only), updates m and l in the exp2 domain with
+//     the scale folded in (scale * log2 e), writes P (fp16 / bf16) back to
+//     TMEM, rescales its O row when m grew, and at the end normalises O by l,
+//     stages it in shared memory (swizzled) and TMA-stores it, and writes LSE.
+//   * The two query tiles ping-pong: while one warpgroup computes its
+//     softmax the tensor core works on the other tile.
+//   * Every mbarrier wait is bounded (globaltimer); a wait that runs past the
+//     limit sets a device error word, the CTA drains its copies and MMAs,
+//     frees TMEM and returns.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "fa_fwd.h"
+
+#define FA_VERSION 10000
+
+namespace fa {
+
+// ----------------------------------------------------------------------------- constants
+
+constexpr int BM = 128;             // query rows per tile (one TMEM lane per row)
+constexpr int BN = 128;             // keys per K / V tile
+constexpr int NQ = 2;               // query tiles per work unit (ping-pong)
+constexpr int UNIT_ROWS = NQ * BM;  // 256
+constexpr int NUM_THREADS = 320;    // warps 0-7 softmax, 8 load, 9 MMA
+constexpr int LOAD_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr int TMEM_COLS = 512;
+constexpr int BOX_BYTES = BM * 128;  // one 128-row x 64-element (128-byte) TMA box
+
+template <int D>
+struct Cfg {
+  static constexpr int TILE_BYTES = BM * D * 2;             // one Q / K / V / O tile
+  static constexpr int NSLOT = (D == 128) ? 5 : 8;           // K / V ring slots
+  static constexpr int NBOX = D / 64;                        // 128-byte boxes per row
+  // mbarrier indices
+  static constexpr int KV_FULL = 0;
+  static constexpr int KV_EMPTY = NSLOT;
+  static constexpr int Q_FULL = 2 * NSLOT;
+  static constexpr int Q_EMPTY = Q_FULL + NQ;
+  static constexpr int S_FULL = Q_EMPTY + NQ;
+  static constexpr int P_FULL = S_FULL + NQ;
+  static constexpr int O_FULL = P_FULL + NQ;
+  static constexpr int O_EMPTY = O_FULL + NQ;
+  static constexpr int EPI = O_EMPTY + NQ;
+  static constexpr int DRAIN = EPI + NQ;
+  static constexpr int NBAR = DRAIN + 1;
+  static constexpr int SMEM_Q = 0;
+  static constexpr int SMEM_KV = NQ * TILE_BYTES;
+  static constexpr int SMEM_BAR = SMEM_KV + NSLOT * TILE_BYTES;
+  static constexpr int SMEM_MISC = SMEM_BAR + NBAR * 8;       // tmem address, abort flag
+  static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;    // + slack for 1024-byte alignment
+};
+
+struct Params {
+  float* lse;
+  int B, H, Sq, Sk;
+  int nqb;             // query units per head: ceil(Sq / 256)
+  int tk;              // key tiles: ceil(Sk / 128)
+  int bh;              // B * H
+  int group_heads;     // heads per L2 group of the schedule
+  int total_units;     // bh * nqb
+  int causal;
+  int bhsd;            // 1: [B,H,S,D], 0: [B,S,H,D]
+  float scale_log2;    // scale * log2(e)
+  unsigned long long wait_limit_ns;
+};
+
+__device__ int g_dev_error = 0;
+
+// ----------------------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase of the given parity.  Returns false (for the
+// whole warp) if the CTA was aborted or the limit ran out; the first warp to
+// run out records the timeout in the device error word.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         uint64_t limit_ns) {
+  bool ok = mbar_try_wait(bar, parity);
+  if (!ok) {
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+      for (int i = 0; i < 16 && !ok; ++i) ok = mbar_try_wait(bar, parity);
+      if (ok) break;
+      if (*abort_flag) break;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        atomicExch(&g_dev_error, 1);
+        break;
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait used only while draining (ignores the abort flag).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) {
+      atomicExch(&g_dev_error, 1);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void tma_store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// tcgen05 -------------------------------------------------------------------
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// D(tmem) (+)= A(smem desc) * B(smem desc)
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D(tmem) (+)= A(tmem) * B(smem desc)
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 lanes x 32 columns of 32-bit words: thread i of the warp gets lane
+// (warp quadrant * 32 + i), columns [col, col + 32).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+        "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+        "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]),
+      "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]),
+      "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Keeps every use of r after the preceding tcgen05.wait::ld (both are volatile asm).
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (BF16) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+// ----------------------------------------------------------------------------- descriptors
+
+// Shared-memory matrix descriptor (sm_100 format): start, leading and stride
+// byte offsets (>> 4), version 1 at bit 46, 128-byte swizzle (2) at bits 61-63.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, A and B of the same
+// 16-bit type (0 fp16, 1 bf16), A K-major, B K-major (0) or MN-major (1).
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, uint32_t fmt, uint32_t b_mn_major) {
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | (b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+// ----------------------------------------------------------------------------- schedule
+
+struct Unit {
+  int b, h, r0;     // batch, head, first query row of the unit
+  int rows[NQ];     // valid rows of each query tile
+  int n[NQ];        // key tiles each query tile visits (0: tile inactive)
+};
+
+// Units are grouped by heads so that the K / V of a group stay in L2; inside
+// a group the longest units (causal: the last query rows) come first.
+__device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
+  const int per_group = p.group_heads * p.nqb;
+  const int g = u / per_group;
+  const int r = u - g * per_group;
+  const int gs = min(p.group_heads, p.bh - g * p.group_heads);
+  const int level = r / gs;
+  const int bh = g * p.group_heads + (r - level * gs);
+  const int qblk = p.causal ? (p.nqb - 1 - level) : level;
+  Unit un;
+  un.b = bh / p.H;
+  un.h = bh - un.b * p.H;
+  un.r0 = qblk * UNIT_ROWS;
+#pragma unroll
+  for (int t = 0; t < NQ; ++t) {
+    const int first = un.r0 + t * BM;
+    const int rows = max(0, min(BM, p.Sq - first));
+    un.rows[t] = rows;
+    if (rows == 0) {
+      un.n[t] = 0;
+    } else if (p.causal) {
+      const int last_key = min(first + rows - 1, p.Sk - 1);
+      un.n[t] = last_key / BN + 1;
+    } else {
+      un.n[t] = p.tk;
+    }
+  }
+  return un;
+}
+
+// ----------------------------------------------------------------------------- kernel
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    fa_fwd_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmQ,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmO) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sQ = smem_u32(smem + C::SMEM_Q);
+  const uint32_t sKV = smem_u32(smem + C::SMEM_KV);
+  const uint32_t bars = smem_u32(smem + C::SMEM_BAR);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint64_t limit = p.wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(bar(C::KV_FULL + s), 1);
+      mbar_init(bar(C::KV_EMPTY + s), 1);
+    }
+    for (int t = 0; t < NQ; ++t) {
+      mbar_init(bar(C::Q_FULL + t), 1);
+      mbar_init(bar(C::Q_EMPTY + t), 1);
+      mbar_init(bar(C::S_FULL + t), 1);
+      mbar_init(bar(C::P_FULL + t), BM);
+      mbar_init(bar(C::O_FULL + t), 1);
+      mbar_init(bar(C::O_EMPTY + t), BM);
+      mbar_init(bar(C::EPI + t), BM);
+    }
+    mbar_init(bar(C::DRAIN), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  constexpr uint32_t FMT = BF16 ? 1u : 0u;
+  constexpr uint32_t IDESC_QK = idesc_f16(BM, BN, FMT, 0);
+  constexpr uint32_t IDESC_PV = idesc_f16(BM, D, FMT, 1);
+
+  if (warp == LOAD_WARP) {
+    // ------------------------------------------------------------------ TMA producer
+    uint32_t kv_cnt = 0;
+    uint32_t q_use[NQ] = {0, 0};
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+      const Unit un = decode_unit(p, u);
+      const int n = max(un.n[0], un.n[1]);
+      for (int t = 0; t < NQ && ok; ++t) {
+        if (un.n[t] == 0) continue;
+        ok = wait_bar(bar(C::Q_EMPTY + t), (q_use[t] & 1u) ^ 1u, abort_flag, limit);
+        if (!ok) break;
+        ++q_use[t];
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar(C::Q_FULL + t), C::TILE_BYTES);
+          const int s0 = un.r0 + t * BM;
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_4d(sQ + t * C::TILE_BYTES + bx * BOX_BYTES, &tmQ, bar(C::Q_FULL + t), bx * 64,
+                        p.bhsd ? s0 : un.h, p.bhsd ? un.h : s0, un.b);
+        }
+        __syncwarp();
+      }
+      for (int j = 0; j < n && ok; ++j) {
+        for (int kv = 0; kv < 2; ++kv) {
+          const uint32_t slot = kv_cnt % C::NSLOT;
+          const uint32_t use = kv_cnt / C::NSLOT;
+          ok = wait_bar(bar(C::KV_EMPTY + slot), (use & 1u) ^ 1u, abort_flag, limit);
+          if (!ok) break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(bar(C::KV_FULL + slot), C::TILE_BYTES);
+            const CUtensorMap* map = kv ? &tmV : &tmK;
+            const int s0 = j * BN;
+            for (int bx = 0; bx < C::NBOX; ++bx)
+              tma_load_4d(sKV + slot * C::TILE_BYTES + bx * BOX_BYTES, map, bar(C::KV_FULL + slot),
+                          bx * 64, p.bhsd ? s0 : un.h, p.bhsd ? un.h : s0, un.b);
+          }
+          __syncwarp();
+          ++kv_cnt;
+        }
+      }
+    }
+    // Drain: wait until every load this warp issued has landed.
+    if (lane == 0) {
+      const uint32_t first = kv_cnt > (uint32_t)C::NSLOT ? kv_cnt - C::NSLOT : 0u;
+      for (uint32_t c = first; c < kv_cnt; ++c)
+        drain_wait(bar(C::KV_FULL + c % C::NSLOT), (c / C::NSLOT) & 1u, limit);
+      for (int t = 0; t < NQ; ++t)
+        if (q_use[t]) drain_wait(bar(C::Q_FULL + t), (q_use[t] - 1) & 1u, limit);
+    }
+    __syncwarp();
+  } else if (warp == MMA_WARP) {
+    // ------------------------------------------------------------------ MMA issuer
+    uint32_t kv_cnt = 0;
+    uint32_t q_use[NQ] = {0, 0}, p_use[NQ] = {0, 0}, o_use[NQ] = {0, 0};
+    bool ok = true;
+    const uint32_t tS0 = tmem, tS1 = tmem + BM;
+    const uint32_t tO0 = tmem + 2 * BM, tO1 = tmem + 2 * BM + D;
+    for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+      const Unit un = decode_unit(p, u);
+      const int n = max(un.n[0], un.n[1]);
+      for (int t = 0; t < NQ && ok; ++t) {
+        if (un.n[t] == 0) continue;
+        ok = wait_bar(bar(C::Q_FULL + t), q_use[t] & 1u, abort_flag, limit);
+        ++q_use[t];
+      }
+      if (!ok) break;
+      // S_t = Q_t K_0^T
+      uint32_t kslot = kv_cnt % C::NSLOT;
+      ok = wait_bar(bar(C::KV_FULL + kslot), (kv_cnt / C::NSLOT) & 1u, abort_flag, limit);
+      if (!ok) break;
+      ++kv_cnt;
+      tc_fence_after();
+      if (lane == 0) {
+        for (int t = 0; t < NQ; ++t) {
+          if (un.n[t] == 0) continue;
+          const uint32_t qa = sQ + t * C::TILE_BYTES, ka = sKV + kslot * C::TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
+            mma_ss(t ? tS1 : tS0, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), IDESC_QK,
+                   kk > 0);
+          }
+          tc_commit(bar(C::S_FULL + t));
+        }
+        tc_commit(bar(C::KV_EMPTY + kslot));
+      }
+      __syncwarp();
+      for (int j = 0; j < n && ok; ++j) {
+        const uint32_t vslot = kv_cnt % C::NSLOT;
+        ok = wait_bar(bar(C::KV_FULL + vslot), (kv_cnt / C::NSLOT) & 1u, abort_flag, limit);
+        if (!ok) break;
+        ++kv_cnt;
+        const bool next_k = (j + 1 < n);
+        bool k_ready = false;
+        kslot = kv_cnt % C::NSLOT;
+        for (int t = 0; t < NQ && ok; ++t) {
+          if (j >= un.n[t]) continue;
+          ok = wait_bar(bar(C::P_FULL + t), p_use[t] & 1u, abort_flag, limit);
+          if (!ok) break;
+          ++p_use[t];
+          if (j == 0) {
+            ok = wait_bar(bar(C::O_EMPTY + t), (o_use[t] & 1u) ^ 1u, abort_flag, limit);
+            if (!ok) break;
+            ++o_use[t];
+          }
+          tc_fence_after();
+          // O_t += P_t V_j   (P_t in TMEM, 16 keys = 8 packed columns per step)
+          if (lane == 0) {
+            const uint32_t va = sKV + vslot * C::TILE_BYTES;
+            const uint32_t tS = t ? tS1 : tS0;
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk)
+              mma_ts(t ? tO1 : tO0, tS + kk * 8, sdesc(va + kk * 2048, BOX_BYTES, 1024), IDESC_PV,
+                     (j > 0 || kk > 0));
+            tc_commit(bar(C::O_FULL + t));
+          }
+          __syncwarp();
+          if (j + 1 < un.n[t]) {
+            if (!k_ready) {
+              ok = wait_bar(bar(C::KV_FULL + kslot), (kv_cnt / C::NSLOT) & 1u, abort_flag, limit);
+              if (!ok) break;
+              ++kv_cnt;
+              k_ready = true;
+              tc_fence_after();
+            }
+            // S_t = Q_t K_{j+1}^T
+            if (lane == 0) {
+              const uint32_t qa = sQ + t * C::TILE_BYTES, ka = sKV + kslot * C::TILE_BYTES;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
+                mma_ss(t ? tS1 : tS0, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), IDESC_QK,
+                       kk > 0);
+              }
+              tc_commit(bar(C::S_FULL + t));
+            }
+            __syncwarp();
+          }
+        }
+        if (!ok) break;
+        if (next_k && !k_ready) {  // cannot happen (n is the max over the tiles); keeps the ring in step
+          ok = wait_bar(bar(C::KV_FULL + kslot), (kv_cnt / C::NSLOT) & 1u, abort_flag, limit);
+          if (!ok) break;
+          ++kv_cnt;
+          k_ready = true;
+        }
+        if (lane == 0) {
+          tc_commit(bar(C::KV_EMPTY + vslot));
+          if (k_ready) tc_commit(bar(C::KV_EMPTY + kslot));
+        }
+        __syncwarp();
+      }
+    }
+    // Drain: every MMA this thread issued has completed before TMEM is freed.
+    if (lane == 0) {
+      tc_commit(bar(C::DRAIN));
+      drain_wait(bar(C::DRAIN), 0, limit);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int t = warp >> 2;               // query tile of this warpgroup
+    const int quad = warp & 3;             // TMEM lane quadrant
+    const int rit = quad * 32 + lane;      // row inside the tile
+    const uint32_t lane_bits = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_bits + t * BM;
+    const uint32_t tO = tmem + lane_bits + 2 * BM + t * D;
+    const float c = p.scale_log2;
+    const bool c_neg = c < 0.f;
+    uint32_t s_use = 0, o_use = 0, e_use = 0;
+    bool ok = true;
+    uint8_t* sQt = smem + C::SMEM_Q + t * C::TILE_BYTES;
+
+    for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+      const Unit un = decode_unit(p, u);
+      const int nt = un.n[t];
+      if (nt == 0) continue;
+      const int row = un.r0 + t * BM + rit;          // query row of this thread
+      const int first_row = un.r0 + t * BM;
+      float m = -INFINITY;                           // running max, log2 domain
+      float l = 0.f;                                 // running exp-sum
+      float m_use = 0.f;
+      for (int j = 0; j < nt; ++j) {
+        ok = wait_bar(bar(C::S_FULL + t), s_use & 1u, abort_flag, limit);
+        if (!ok) break;
+        ++s_use;
+        tc_fence_after();
+        float s[BN];
+        {
+          uint32_t r[32];
+#pragma unroll
+          for (int q4 = 0; q4 < BN / 32; ++q4) {
+            tmem_ld32(tS + q4 * 32, r);
+            tmem_wait_ld();
+            reg_fence(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[q4 * 32 + i] = __uint_as_float(r[i]);
+          }
+        }
+        const int c0 = j * BN;
+        const bool tail = (c0 + BN > p.Sk);
+        const bool diag = p.causal && (c0 + BN - 1 > first_row);
+        float cc = c;
+        float m_blk;
+        if (tail || diag) {
+          // masked tile: work on scaled logits, masked entries -> -inf
+          int lim = p.Sk - 1 - c0;
+          if (p.causal) lim = min(lim, row - c0);
+          float mx = -INFINITY;
+#pragma unroll
+          for (int k = 0; k < BN; ++k) {
+            const float tv = (k > lim) ? -INFINITY : s[k] * c;
+            s[k] = tv;
+            mx = fmaxf(mx, tv);
+          }
+          m_blk = mx;
+          cc = 1.f;
+        } else if (!c_neg) {
+          float a0 = s[0], a1 = s[1], a2 = s[2], a3 = s[3];
+#pragma unroll
+          for (int k = 4; k < BN; k += 4) {
+            a0 = fmaxf(a0, s[k]);
+            a1 = fmaxf(a1, s[k + 1]);
+            a2 = fmaxf(a2, s[k + 2]);
+            a3 = fmaxf(a3, s[k + 3]);
+          }
+          m_blk = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * c;
+        } else {
+          float a0 = s[0], a1 = s[1], a2 = s[2], a3 = s[3];
+#pragma unroll
+          for (int k = 4; k < BN; k += 4) {
+            a0 = fminf(a0, s[k]);
+            a1 = fminf(a1, s[k + 1]);
+            a2 = fminf(a2, s[k + 2]);
+            a3 = fminf(a3, s[k + 3]);
+          }
+          m_blk = fminf(fminf(a0, a1), fminf(a2, a3)) * c;
+        }
+        const float m_new = fmaxf(m, m_blk);
+        m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        const float alpha = ex2(m - m_use);          // 0 on the first tile, 1 if m did not grow
+        m = m_new;
+        const float neg_m = -m_use;
+        float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int k = 0; k < BN; k += 4) {
+          const float p0 = ex2(fmaf(s[k], cc, neg_m));
+          const float p1 = ex2(fmaf(s[k + 1], cc, neg_m));
+          const float p2 = ex2(fmaf(s[k + 2], cc, neg_m));
+          const float p3 = ex2(fmaf(s[k + 3], cc, neg_m));
+          rs0 += p0;
+          rs1 += p1;
+          rs2 += p2;
+          rs3 += p3;
+          pk[k / 2] = pack2<BF16>(p0, p1);
+          pk[k / 2 + 1] = pack2<BF16>(p2, p3);
+        }
+        l = l * alpha + ((rs0 + rs1) + (rs2 + rs3));
+        // P_t -> TMEM (first 64 columns of S_t)
+        {
+          uint32_t r[32];
+#pragma unroll
+          for (int h2 = 0; h2 < BN / 64; ++h2) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = pk[h2 * 32 + i];
+            tmem_st32(tS + h2 * 32, r);
+          }
+        }
+        if (j > 0) {
+          // O_t of the previous tile is complete; rescale it if any row's max grew
+          ok = wait_bar(bar(C::O_FULL + t), o_use & 1u, abort_flag, limit);
+          if (!ok) break;
+          ++o_use;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            uint32_t r[32];
+#pragma unroll
+            for (int q4 = 0; q4 < D / 32; ++q4) {
+              tmem_ld32(tO + q4 * 32, r);
+              tmem_wait_ld();
+              reg_fence(r);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+              tmem_st32(tO + q4 * 32, r);
+            }
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::P_FULL + t));
+      }
+      if (!ok) break;
+
+      // ---------------------------------------------------------------- epilogue
+      ok = wait_bar(bar(C::O_FULL + t), o_use & 1u, abort_flag, limit);
+      if (!ok) break;
+      ++o_use;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      {
+        uint32_t r[32];
+#pragma unroll
+        for (int q4 = 0; q4 < D / 32; ++q4) {
+          tmem_ld32(tO + q4 * 32, r);
+          tmem_wait_ld();
+          reg_fence(r);
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
+          // row rit of box q4/2, 16-byte chunks (q4&1)*4 + i, 128-byte swizzle
+          uint8_t* rowp = sQt + (q4 >> 1) * BOX_BYTES + rit * 128;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int chunk = ((q4 & 1) * 4 + i) ^ (rit & 7);
+            *reinterpret_cast<uint4*>(rowp + chunk * 16) = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::O_EMPTY + t));
+      fence_proxy_async_smem();
+      mbar_arrive(bar(C::EPI + t));
+      if (row < p.Sq) {
+        const float lse = (m_use + lg2(l)) * 0.69314718055994530942f;
+        p.lse[((size_t)(un.b * p.H + un.h)) * p.Sq + row] = lse;
+      }
+      if (rit == 0) {
+        // one thread stores the tile once all 128 rows are staged
+        drain_wait(bar(C::EPI + t), e_use & 1u, limit);
+        const int s0 = first_row;
+        for (int bx = 0; bx < C::NBOX; ++bx)
+          tma_store_4d(&tmO, smem_u32(sQt + bx * BOX_BYTES), bx * 64, p.bhsd ? s0 : un.h,
+                       p.bhsd ? un.h : s0, un.b);
+        tma_store_commit();
+        tma_store_wait_read();
+        mbar_arrive(bar(C::Q_EMPTY + t));
+      }
+      ++e_use;
+      __syncwarp();
+    }
+    if (rit == 0) tma_store_wait_all();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace fa
+
+// ============================================================================= host side
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+fa_status cuda_fail(int err) {
+  t_last_cuda_error = err;
+  return FA_ERR_CUDA;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn(int* err) {
+  static EncodeTiledFn fn = nullptr;
+  static int init_err = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !ptr) {
+      init_err = (e != cudaSuccess) ? (int)e : 999;
+      return;
+    }
+    fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  *err = init_err;
+  return fn;
+}
+
+// A [B, S, H, D] (BSND) or [B, H, S, D] (BHSD) tensor seen as 4-D for TMA,
+// dims in memory order, 128-row x 64-column boxes with a 128-byte swizzle.
+fa_status make_map(CUtensorMap* map, const void* base, fa_dtype dt, fa_layout lay, int64_t B, int64_t H,
+                   int64_t S, int64_t D) {
+  int err = 0;
+  EncodeTiledFn enc = get_encode_fn(&err);
+  if (!enc) return cuda_fail(err);
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4];
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  if (lay == FA_BHSD) {
+    dims[0] = D; dims[1] = S; dims[2] = H; dims[3] = B;
+    strides[0] = D * 2; strides[1] = S * D * 2; strides[2] = H * S * D * 2;
+    box[0] = 64; box[1] = fa::BM; box[2] = 1; box[3] = 1;
+  } else {
+    dims[0] = D; dims[1] = H; dims[2] = S; dims[3] = B;
+    strides[0] = D * 2; strides[1] = H * D * 2; strides[2] = S * H * D * 2;
+    box[0] = 64; box[1] = 1; box[2] = fa::BM; box[3] = 1;
+  }
+  const CUtensorMapDataType t =
+      dt == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = enc(map, t, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail((int)r);
+  return FA_OK;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+fa_status check_device_ptr(const void* ptr, int device) {
+  cudaPointerAttributes attr;
+  cudaError_t e = cudaPointerGetAttributes(&attr, ptr);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail((int)e);
+  }
+  if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return FA_ERR_NOT_DEVICE_POINTER;
+  if (attr.device != device) return FA_ERR_NOT_DEVICE_POINTER;
+  return FA_OK;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  bool configured[4] = {false, false, false, false};
+};
+
+template <int D, bool BF16>
+fa_status launch(const fa::Params& prm, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                 const CUtensorMap& o, int grid, bool* configured, cudaStream_t stream) {
+  auto kern = fa::fa_fwd_kernel<D, BF16>;
+  const int smem = fa::Cfg<D>::SMEM_BYTES;
+  if (!*configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail((int)e);
+    *configured = true;
+  }
+  kern<<<grid, fa::NUM_THREADS, smem, stream>>>(prm, q, k, v, o);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail((int)e);
+  return FA_OK;
+}
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                 int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
+                 void* stream) {
+  // ---- arguments that need no device
+  if (B <= 0 || H <= 0 || Sq < 0 || Sk <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
+  if (layout != FA_BSND && layout != FA_BHSD) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  // TMA coordinates and the schedule use 32-bit integers
+  const int64_t lim = (int64_t)1 << 30;
+  if (B >= lim || H >= lim || Sq >= lim || Sk >= lim || B * H >= lim) return FA_ERR_UNSUPPORTED;
+  const int64_t nqb = (Sq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+  if (B * H * nqb >= lim) return FA_ERR_UNSUPPORTED;
+  if (Sq == 0) return FA_OK;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
+       reinterpret_cast<uintptr_t>(o)) & 15u)
+    return FA_ERR_MISALIGNED;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA_ERR_MISALIGNED;
+  const size_t qbytes = (size_t)(B * H * Sq * D) * 2, kvbytes = (size_t)(B * H * Sk * D) * 2;
+  const size_t lbytes = (size_t)(B * H * Sq) * 4;
+  if (overlaps(o, qbytes, q, qbytes) || overlaps(o, qbytes, k, kvbytes) || overlaps(o, qbytes, v, kvbytes) ||
+      overlaps(lse, lbytes, q, qbytes) || overlaps(lse, lbytes, k, kvbytes) ||
+      overlaps(lse, lbytes, v, kvbytes) || overlaps(lse, lbytes, o, qbytes))
+    return FA_ERR_ALIAS;
+
+  // ---- device checks
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail((int)e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  const void* ptrs[5] = {q, k, v, o, lse};
+  for (const void* ptr : ptrs) {
+    fa_status st = check_device_ptr(ptr, dev);
+    if (st != FA_OK) return st;
+  }
+  int sms;
+  {
+    std::lock_guard<std::mutex> g(g_dev_mu);
+    if (g_dev[dev].sms == 0) {
+      e = cudaDeviceGetAttribute(&g_dev[dev].sms, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return cuda_fail((int)e);
+    }
+    sms = g_dev[dev].sms;
+  }
+
+  CUtensorMap mq, mk, mv, mo;
+  fa_status st;
+  if ((st = make_map(&mq, q, dtype, layout, B, H, Sq, D)) != FA_OK) return st;
+  if ((st = make_map(&mk, k, dtype, layout, B, H, Sk, D)) != FA_OK) return st;
+  if ((st = make_map(&mv, v, dtype, layout, B, H, Sk, D)) != FA_OK) return st;
+  if ((st = make_map(&mo, o, dtype, layout, B, H, Sq, D)) != FA_OK) return st;
+
+  fa::Params prm;
+  prm.lse = lse;
+  prm.B = (int)B;
+  prm.H = (int)H;
+  prm.Sq = (int)Sq;
+  prm.Sk = (int)Sk;
+  prm.nqb = (int)nqb;
+  prm.tk = (int)((Sk + fa::BN - 1) / fa::BN);
+  prm.bh = (int)(B * H);
+  // heads whose K and V fit together in about 48 MB of L2
+  const int64_t kv_head_bytes = 2 * Sk * D * 2;
+  int64_t gh = ((int64_t)48 << 20) / (kv_head_bytes > 0 ? kv_head_bytes : 1);
+  if (gh < 1) gh = 1;
+  if (gh > B * H) gh = B * H;
+  prm.group_heads = (int)gh;
+  prm.total_units = (int)(B * H * nqb);
+  prm.causal = causal ? 1 : 0;
+  prm.bhsd = layout == FA_BHSD ? 1 : 0;
+  prm.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  prm.wait_limit_ns = 1000000000ull;  // one second; a normal wait lasts microseconds
+
+  const int grid = (int)(prm.total_units < sms ? prm.total_units : sms);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bool* cfg = g_dev[dev].configured;
+  if (D == 128)
+    return dtype == FA_BF16 ? launch<128, true>(prm, mq, mk, mv, mo, grid, &cfg[0], s)
+                            : launch<128, false>(prm, mq, mk, mv, mo, grid, &cfg[1], s);
+  return dtype == FA_BF16 ? launch<64, true>(prm, mq, mk, mv, mo, grid, &cfg[2], s)
+                          : launch<64, false>(prm, mq, mk, mv, mo, grid, &cfg[3], s);
+}
+
+fa_status fa_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail((int)e);
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, fa::g_dev_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail((int)e);
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(fa::g_dev_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail((int)e);
+    return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}
+
+fa_status fa_query_support(int64_t D, fa_dtype dtype) {
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+  return (D == 64 || D == 128) ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+const char* fa_status_string(fa_status status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_NOT_DEVICE_POINTER: return "FA_ERR_NOT_DEVICE_POINTER";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED";
+    case FA_ERR_ALIAS: return "FA_ERR_ALIAS";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+int fa_last_cuda_error(void) { return t_last_cuda_error; }
+
+int fa_version(void) { return FA_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,141 @@
+/*
+ * fa_fwd.h -- C ABI of the B200 (sm_100a) FlashAttention forward library,
+ * libfa_fwd.so.
+ *
+ * The operation.  For every batch b, head h and query row i
+ *
+ *     O[b,h,i,:] = softmax_j( scale * q[b,h,i,:] . k[b,h,j,:]  [+ causal mask] ) * V[b,h,:,:]
+ *     LSE[b,h,i] = ln( sum_j exp( scale * q[b,h,i,:] . k[b,h,j,:] ) )   over the visible keys j
+ *
+ * computed tile by tile with an online softmax (running row max and running
+ * exp-sum, rescaled per key/value tile) so that the Sq x Sk score matrix never
+ * reaches device memory.  Sources on the pages:
+ *   - the standard attention it must equal, and the tiling + online-softmax
+ *     method: page "FlashAttention: long-text inference without running out
+ *     of memory" (ai6s.net/6a0d42d8), sections "the memory black hole" and
+ *     "FlashAttention's answer: tiling + online normalisation";
+ *   - the causal flag in place of a mask tensor: page "FlashAttention in
+ *     ops-transformer on Ascend NPU" (ai6s.net/6a0d3bfb), section "how
+ *     FlashAttention runs on the Ascend NPU" (causal=True, not a triu mask);
+ *   - whole-tile skipping above the diagonal: page "catlass FlashAttention
+ *     template tuning" (hwcomputing.csdn.net/6a0d4681), section "causal mask
+ *     implementations", mode 2 (diagonal skip);
+ *   - the per-row log-sum-exp [B, H, S] in natural log: page "64K
+ *     long-sequence FlashAttention" (ai6s.net/6a140d07), section "layer 2:
+ *     numerical stability";
+ *   - the call shape flash_attention(q, k, v, head_num, input_layout, scale)
+ *     and the BSND / BNSD layouts: page "ops-transformer FlashAttention on
+ *     Atlas 800" (hwcomputing.csdn.net/6a0d4444), sections "minimal runnable
+ *     code" and the error table; page hwcomputing.csdn.net/6a0d4681, section
+ *     "data layout";
+ *   - fp16 and bf16 as the two half-precision choices: page
+ *     hwcomputing.csdn.net/6a0d4681, section "precision choice".
+ *
+ * Causal masking is aligned at the top-left corner: key j is visible to query
+ * i iff j <= i (the pages only show the square case, triu(ones(S,S), 1)).
+ * Every row therefore sees at least key 0.
+ *
+ * Arithmetic: q.k products accumulate in fp32 on the tensor cores; the
+ * softmax runs in fp32; the probabilities are rounded to the input dtype
+ * before P.V (fp32 accumulation); O is rounded to the input dtype once, at
+ * the end; LSE is fp32.
+ */
+#ifndef FA_FWD_H
+#define FA_FWD_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes.  No entry point crashes on a bad argument: it returns one of these. */
+typedef enum fa_status {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,        /* null pointer, non-positive size, bad enum, non-finite scale, Sk = 0 */
+    FA_ERR_UNSUPPORTED = 2,        /* head dim D not in {64, 128}, or a size beyond the 32-bit tile coordinates */
+    FA_ERR_NOT_DEVICE_POINTER = 3, /* a tensor pointer is host memory (the pages: a CPU tensor segfaults; here it is refused) */
+    FA_ERR_MISALIGNED = 4,         /* q, k, v or o not 16-byte aligned (TMA), or lse not 4-byte aligned */
+    FA_ERR_ALIAS = 5,              /* o or lse overlaps q, k or v, or o overlaps lse */
+    FA_ERR_CUDA = 6,               /* a CUDA runtime / driver call failed; see fa_last_cuda_error() */
+    FA_ERR_TIMEOUT = 7             /* a kernel wait ran past its limit (reported by fa_device_status) */
+} fa_status;
+
+/* Tensor layouts.  "N" is the head axis: BSND == BSHD, BHSD == BNSD. */
+typedef enum fa_layout {
+    FA_BSND = 0,   /* q: [B, Sq, H, D], k and v: [B, Sk, H, D], o like q */
+    FA_BHSD = 1    /* q: [B, H, Sq, D], k and v: [B, H, Sk, D], o like q */
+} fa_layout;
+
+/* Element type of q, k, v and o. */
+typedef enum fa_dtype {
+    FA_FP16 = 0,
+    FA_BF16 = 1
+} fa_dtype;
+
+/*
+ * fa_fwd -- the attention forward pass, asynchronous on `stream`.
+ *
+ * q, k, v   device pointers, dense and contiguous in `layout` (row-major,
+ *           innermost axis D), element type `dtype`; read only.  16-byte
+ *           aligned (they are read with TMA).
+ * o         device pointer, same shape, layout and dtype as q; every element
+ *           is overwritten.  16-byte aligned.
+ * lse       device pointer to B*H*Sq fp32 values laid out [B, H, Sq]
+ *           (head-major in both layouts); every element is overwritten with
+ *           the natural-log log-sum-exp of the row's scaled, masked logits.
+ * B, H      batch and head counts (>= 1).
+ * Sq, Sk    query and key lengths.  Sq = 0 is a no-op returning FA_OK; Sk must
+ *           be >= 1 (a softmax over no keys is undefined).  Neither needs to be
+ *           a multiple of the tile: ragged tails are masked in the kernel.
+ * D         head dimension, 64 or 128.
+ * layout    FA_BSND or FA_BHSD.
+ * causal    non-zero: key j is visible to query i iff j <= i.
+ * scale     multiplies q.k before the softmax, used as given (any finite
+ *           value, 0 included; the usual choice is 1/sqrt(D)).
+ * dtype     FA_FP16 or FA_BF16.
+ * stream    a cudaStream_t (passed as void*); NULL is the legacy default stream.
+ *
+ * Ownership: the caller allocates and owns every buffer; the library keeps no
+ * pointer after the call returns and allocates no device memory.  o and lse
+ * must not overlap q, k, v or each other.
+ *
+ * Errors: arguments are validated before anything is launched and every
+ * failure is a return code.  FA_ERR_CUDA means a launch or driver call
+ * failed; fa_last_cuda_error() gives the CUDA error number.  A kernel whose
+ * internal wait exceeded its limit (which indicates a bug, never expected)
+ * stops early, leaves o / lse unspecified, and is reported by the next
+ * fa_device_status() call.
+ *
+ * The call does not synchronise.  It is safe to call from several host
+ * threads on different streams.
+ */
+fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+                 int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D,
+                 fa_layout layout, int causal, float scale, fa_dtype dtype, void *stream);
+
+/*
+ * fa_device_status -- synchronises `stream`, then reads and clears the
+ * library's device-side error word on the current device.  Returns FA_OK,
+ * FA_ERR_TIMEOUT if a kernel stopped at a wait limit since the last call, or
+ * FA_ERR_CUDA if the synchronisation itself failed.
+ */
+fa_status fa_device_status(void *stream);
+
+/* FA_OK if (D, dtype) is supported by fa_fwd, FA_ERR_UNSUPPORTED otherwise. */
+fa_status fa_query_support(int64_t D, fa_dtype dtype);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *fa_status_string(fa_status status);
+
+/* The cudaError_t / CUresult number behind the last FA_ERR_CUDA on this host thread (0 if none). */
+int fa_last_cuda_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_FWD_H */

@@ -1,0 +1,133 @@
+"""CPU tests of the C ABI: the library loads, exports every function the header
+declares, and rejects bad arguments before touching the GPU.
+
+Only argument checks that return before the first CUDA call are exercised
+here (fake, never-dereferenced pointer values); everything that needs a
+device is in the gpu-marked tests.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import attention_forward_19_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa_fwd.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return fa.load_library()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names, "no declarations found in the header"
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in fa_fwd.h but not exported"
+    assert sorted(fa.EXPORTED_SYMBOLS) == names
+
+
+def test_exported_symbols_are_plain_c(lib):
+    # nm-free check: the C names resolve through dlsym, i.e. they are not mangled
+    for name in declared_functions():
+        ctypes.cast(getattr(lib, name), ctypes.c_void_p)
+
+
+def test_version_and_strings(lib):
+    assert fa.fa_version() == 10000
+    for code, name in [(0, "FA_OK"), (1, "FA_ERR_INVALID_ARG"), (2, "FA_ERR_UNSUPPORTED"),
+                       (3, "FA_ERR_NOT_DEVICE_POINTER"), (4, "FA_ERR_MISALIGNED"), (5, "FA_ERR_ALIAS"),
+                       (6, "FA_ERR_CUDA"), (7, "FA_ERR_TIMEOUT")]:
+        assert fa.fa_status_string(code) == name
+    assert fa.fa_status_string(99) == "FA_ERR_UNKNOWN"
+    assert fa.fa_last_cuda_error() == 0
+
+
+def test_query_support(lib):
+    for D in (64, 128):
+        for dt in (fa.FA_FP16, fa.FA_BF16):
+            assert fa.fa_query_support(D, dt) == fa.FA_OK
+    for D in (0, 32, 96, 256):
+        assert fa.fa_query_support(D, fa.FA_BF16) == fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_query_support(128, 7) == fa.FA_ERR_UNSUPPORTED
+
+
+# Fake, 256-byte aligned, far-apart addresses: the checks below return before any use.
+Q, K, V, O, L = 0x10000000, 0x20000000, 0x30000000, 0x40000000, 0x50000000
+GOOD = dict(B=1, H=2, Sq=512, Sk=512, D=64, layout=fa.FA_BSND, causal=0, scale=0.125, dtype=fa.FA_FP16)
+
+
+def call(q=Q, k=K, v=V, o=O, lse=L, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_fwd(q, k, v, o, lse, a["B"], a["H"], a["Sq"], a["Sk"], a["D"], a["layout"], a["causal"],
+                     a["scale"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw", [dict(B=0), dict(H=0), dict(B=-1), dict(Sk=0), dict(Sq=-1), dict(D=0),
+                                dict(layout=2), dict(layout=-1), dict(dtype=2),
+                                dict(scale=float("nan")), dict(scale=float("inf"))])
+def test_invalid_arguments(lib, kw):
+    assert call(**kw) == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("D", [32, 80, 96, 256])
+def test_unsupported_head_dim(lib, D):
+    assert call(D=D) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_oversized_lengths_unsupported(lib):
+    assert call(Sq=1 << 31) == fa.FA_ERR_UNSUPPORTED
+    assert call(Sk=1 << 31) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_empty_query_is_a_no_op(lib):
+    assert call(Sq=0) == fa.FA_OK
+    assert call(Sq=0, q=0, o=0, lse=0) == fa.FA_OK
+
+
+@pytest.mark.parametrize("which", ["q", "k", "v", "o", "lse"])
+def test_null_pointer(lib, which):
+    assert call(**{which: 0}) == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("which,off", [("q", 8), ("k", 2), ("v", 4), ("o", 8), ("lse", 2)])
+def test_misaligned_pointer(lib, which, off):
+    base = dict(q=Q, k=K, v=V, o=O, lse=L)[which]
+    assert call(**{which: base + off}) == fa.FA_ERR_MISALIGNED
+
+
+def test_lse_needs_only_4_byte_alignment(lib):
+    # passes the alignment and alias checks; on a machine without a GPU it then fails in CUDA
+    st = call(lse=L + 4)
+    assert st not in (fa.FA_ERR_MISALIGNED, fa.FA_ERR_ALIAS, fa.FA_ERR_INVALID_ARG)
+
+
+@pytest.mark.parametrize("o,lse", [(Q, L), (Q + 4096, L), (K, L), (V + 64, L), (O, Q), (O, O + 16), (O, V)])
+def test_aliasing_outputs_rejected(lib, o, lse):
+    assert call(o=o, lse=lse) == fa.FA_ERR_ALIAS
+
+
+def test_python_wrapper_checks_shapes():
+    torch = pytest.importorskip("torch")
+    q = torch.zeros(1, 16, 2, 64, dtype=torch.float16)
+    k = torch.zeros(1, 16, 3, 64, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        fa.flash_attention_forward(q, k, k, layout="BSND")
+    with pytest.raises(ValueError, match="head_num"):
+        fa.flash_attention_forward(q, q, q, layout="BSND", head_num=8)
+    with pytest.raises(TypeError):
+        x = torch.zeros(1, 16, 2, 64, dtype=torch.float32)
+        fa.flash_attention_forward(x, x, x, layout="BSND")
+    with pytest.raises(ValueError, match="contiguous"):
+        t = torch.zeros(1, 2, 16, 64, dtype=torch.float16).transpose(1, 2)
+        fa.flash_attention_forward(t, t, t, layout="BSND")
