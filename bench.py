@@ -1,0 +1,380 @@
+"""Benchmark of the B200 FlashAttention forward (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {native,reference}]
+
+A step is one attention forward over the workload
+bf16 BHSD B=2 H=40 Sq=Sk=8192 D=128, causal, scale 1/sqrt(128), q/k/v ~ N(0,1).
+The metric is attention-forward TFLOP/s with the causal-halved flop count
+4*B*H*Sq*Sk*D/2.  Timing: W untimed warm-up steps, then exactly K steps
+between a barrier + torch.cuda.synchronize() on both sides, timed with CUDA
+events on the stream the kernel is launched on; with N > 1 ranks (torchrun)
+every rank processes its own full workload (weak scaling, no collective on
+the data path) and the time is the max over ranks.  The inputs (3 x 168 MB)
+are larger than the 126 MB L2, so no flush is done between steps.
+
+--impl reference runs the fp64 CPU oracle (the parity reference) on rank 0
+on a bounded row sample of the same workload, each step one sample.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from fa_inputs import BENCH_WORKLOAD, WORKLOADS, make_qkv  # noqa: E402
+
+METRIC = "attn fwd TFLOP/s (causal-halved) and % of B200 dense fp16/bf16 tensor peak"
+UNIT = "TFLOP/s"
+SPEC_PEAK_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SRC = os.path.join(ROOT, "attention_forward_19_b200", "csrc", "fa_fwd.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "fa_fwd_bf16_bhsd_b2_h40_s8192_d128_causal.dram.json")
+
+
+def kernel_hash():
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def workload_config(w, n_gpus):
+    return {
+        "workload": w.name, "model": "attention forward (no weights)", "B": w.B, "H": w.H, "Sq": w.Sq,
+        "Sk": w.Sk, "D": w.D, "layout": w.layout, "causal": w.causal, "scale": w.scale, "dtype": w.dtype,
+        "global_batch": w.B * n_gpus, "seq_len": w.Sq, "parallelism": f"dp{n_gpus} (independent heads per rank)",
+        "l2": "no flush: inputs 3 x 168 MB > 126 MB L2",
+        "inputs": "seeded N(0,1), fp32 randn rounded to bf16",
+    }
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self._t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+
+def oracle_sample(w, target_s, max_rows=None, threads=0):
+    """Times the fp64 oracle on stratified rows of w for about target_s seconds.
+
+    Returns (tflops, seconds, rows, threads): flops count 4*D per visible (query, key) pair.
+    """
+    import numpy as np
+    from oracle import attn
+    orc = attn.default()
+    q, k, v = make_qkv(w)
+    nthreads = threads if threads > 0 else orc.max_threads()
+    rng = np.random.default_rng(12345)
+    total_rows = w.B * w.H * w.Sq
+    flops = 0.0
+    done = 0
+    t0 = time.perf_counter()
+    batch = 64
+    while True:
+        rows = rng.integers(0, total_rows, size=batch, dtype=np.int64)
+        i = rows % w.Sq
+        vis = np.minimum(i + 1, w.Sk) if w.causal else np.full_like(i, w.Sk)
+        orc.fwd(q, k, v, layout=w.layout, causal=w.causal, scale=float(np.float32(w.scale)), rows=rows,
+                threads=nthreads)
+        flops += float(4.0 * w.D * vis.sum())
+        done += batch
+        el = time.perf_counter() - t0
+        if el >= target_s or (max_rows is not None and done >= max_rows):
+            break
+        batch = min(batch * 2, 8192)
+    return flops / el / 1e12, el, done, nthreads
+
+
+# ----------------------------------------------------------------------------- native arm
+
+
+def bench_workload(args):
+    """The timed workload; --workload / --bh select another one (profiling runs only)."""
+    w = WORKLOADS[args.workload]
+    if args.bh:
+        b, h = (int(x) for x in args.bh.split(","))
+        w = w.with_(B=b, H=h, name=f"{w.name}_b{b}_h{h}")
+    return w
+
+
+def rank_workload(w0, rank):
+    """Weak scaling: every rank runs the full workload on its own inputs (seed offset by rank)."""
+    return w0.with_(seed=w0.seed + 1000 * rank)
+
+
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time (a scalar all-reduce; no data-path collective)."""
+    if world == 1:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_native(args, rank, world, local_rank):
+    import attention_forward_19_b200 as fa
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w0 = bench_workload(args)
+    w = rank_workload(w0, rank)
+    q, k, v = make_qkv(w, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.flash_attention_forward(q, k, v, layout=w.layout, causal=w.causal, scale=w.scale, out=o, lse=lse,
+                                   stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    fa.check_device_status(stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(cvd.split(",")[local_rank].strip() if cvd else str(local_rank))
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    ms_local = e0.elapsed_time(e1)
+    fa.check_device_status(stream)
+    ms_total = max_over_ranks(ms_local, world, dev)
+    ms_step = ms_total / args.steps
+    flops = w.flops()
+    value = world * flops * args.steps / (ms_total * 1e-3) / 1e12
+
+    if args.no_e2e:
+        if rank == 0:
+            print(f"{w.name}: {ms_step:.4f} ms/step, {value:.1f} TFLOP/s (no e2e, no baseline)", flush=True)
+        return None
+    # end to end through the public API: pinned host inputs -> device -> kernel -> host result
+    e2e_steps = max(3, min(args.steps, 10))
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+    def e2e_step():
+        dq = hq.to(dev, non_blocking=True)
+        dk = hk.to(dev, non_blocking=True)
+        dv = hv.to(dev, non_blocking=True)
+        do, dl = fa.flash_attention_forward(dq, dk, dv, layout=w.layout, causal=w.causal, scale=w.scale,
+                                            stream=stream)
+        ho.copy_(do, non_blocking=True)
+        hl.copy_(dl, non_blocking=True)
+
+    e2e_step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(a0.elapsed_time(a1), world, dev)
+    fa.check_device_status(stream)
+    e2e_value = world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    traffic = None
+    traffic_note = "no ncu capture of this kernel version"
+    if os.path.exists(TRAFFIC_FILE):
+        with open(TRAFFIC_FILE) as f:
+            tr = json.load(f)
+        if tr.get("kernel_sha256_16") == kernel_hash():
+            traffic = tr.get("dram_bytes_per_launch")
+            traffic_note = tr.get("note", "")
+        else:
+            traffic_note = "ncu capture is of an older kernel version"
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        tf, secs, nrows, thr = oracle_sample(w0, target_s=args.cpu_seconds)
+        cpu = {"value": tf, "unit": UNIT, "cores": thr, "kind": "oracle",
+               "sample": f"{nrows} random query rows of the same workload (fp64, all their visible keys), "
+                         f"{secs:.1f} s"}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(w0, world),
+        "pct_of_spec_peak": 100.0 * value / world / SPEC_PEAK_TFLOPS,
+        "pct_of_measured_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
+                                    if peak_kind == "measured" else "fallback 1590 TFLOP/s",
+                     "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"]),
+                     "frac_of_spec_2250": achieved / SPEC_PEAK_TFLOPS,
+                     "algorithmic_flops_per_launch": flops, "traffic_note": traffic_note},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "kernel": "fa::fa_fwd_kernel<128, true> (libfa_fwd.so)",
+    }
+    return line
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = bench_workload(args)
+    per_step = max(0.5, args.ref_seconds / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(w, target_s=per_step)
+    vals, secs, rows = [], 0.0, 0
+    thr = None
+    for _ in range(args.steps):
+        tf, s, n, thr = oracle_sample(w, target_s=per_step)
+        vals.append(tf)
+        secs += s
+        rows += n
+    value = statistics.mean(vals)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                         "sample": f"each step: random query rows of the workload for ~{per_step:.1f} s "
+                                   f"({rows} rows in total), fp64"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="time the kernel only (profiling runs)")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default=BENCH_WORKLOAD)
+    ap.add_argument("--bh", default=None, help="override B,H of the workload (profiling runs)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import datetime
+            torch.cuda.set_device(local_rank)
+            torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                                 device_id=torch.device("cuda", local_rank))
+        try:
+            line = run_native(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
