@@ -65,6 +65,14 @@ constexpr int LOAD_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr int TMEM_COLS = 512;
 constexpr int BOX_BYTES = BM * 128;  // one 128-row x 64-element (128-byte) TMA box
+#ifndef FA_RESCALE_LOG2
+#define FA_RESCALE_LOG2 8.0f
+#endif
+constexpr float RESCALE_LOG2 = FA_RESCALE_LOG2;  // O / l are rescaled only when a row max grows by more (log2 units)
+#ifndef FA_EMU_PAIRS
+#define FA_EMU_PAIRS 1
+#endif
+constexpr int EMU_PAIRS = FA_EMU_PAIRS;  // of every 4 exp2 pairs, this many run on the FMA pipe
 
 template <int D>
 struct Cfg {
@@ -167,6 +175,24 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   return __all_sync(0xffffffffu, ok);
 }
 
+// Bounded wait for one thread (the producer and MMA roles run on lane 0 only).
+__device__ __forceinline__ bool wait_bar1(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 16; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicExch(&g_dev_error, 1);
+      return false;
+    }
+  }
+}
+
 // Bounded wait used only while draining (ignores the abort flag).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return;
@@ -232,6 +258,36 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                : "memory");
 }
 
+// The *_elect forms are executed by a whole (converged) warp, so their
+// operands stay warp-uniform; one elected lane issues the instruction.
+__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_elect(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+
 // D(tmem) (+)= A(smem desc) * B(smem desc)
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
@@ -293,6 +349,15 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
+// Columns [col, col + 32 * N) of this warp's 32 lanes into r, one wait for all.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[32 * N]) {
+#pragma unroll
+  for (int c = 0; c < N; ++c) tmem_ld32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+  tmem_wait_ld();
+  reg_fence(r);
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -314,6 +379,137 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
   }
+}
+
+template <bool BF16>
+__device__ __forceinline__ float round_to_input(float x) {
+  if constexpr (BF16) return __bfloat162float(__float2bfloat16_rn(x));
+  else return __half2float(__float2half_rn(x));
+}
+
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction for two lanes of work).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void f2unpack(uint64_t d, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(d));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for two values on the FMA pipe instead of MUFU.  x = j + r with
+// j = round(x): adding 1.5 * 2^23 leaves j in the low mantissa bits, so
+// 1.5 * 2^23 - (x + 1.5 * 2^23) = -j exactly and r = x - j lies in [-1/2, 1/2].
+// 2^r is a polynomial (constant term 1; near-minimax in relative error, fitted
+// by csrc/gen_exp2_poly.py: 1.0e-4 at degree 3, 2.9e-6 at degree 4), and 2^j
+// is added to its exponent field.  x is clamped at -125 so the exponent stays
+// normal; 2^-125 stands in for anything smaller.
+template <int DEG>
+__device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& y0, float& y1) {
+  float x0, x1;
+  f2unpack(x2, x0, x1);
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  const uint64_t magic = f2pack(12582912.f, 12582912.f);
+  const uint64_t t = fadd2(f2pack(x0, x1), magic);
+  const uint64_t neg_j = ffma2(t, f2pack(-1.f, -1.f), magic);
+  const uint64_t r = fadd2(f2pack(x0, x1), neg_j);
+  uint64_t p;
+  if constexpr (DEG == 3) {
+    p = ffma2(r, f2pack(5.500874668e-02f, 5.500874668e-02f), f2pack(2.422107607e-01f, 2.422107607e-01f));
+    p = ffma2(p, r, f2pack(6.932829022e-01f, 6.932829022e-01f));
+  } else {
+    p = ffma2(r, f2pack(9.582836181e-03f, 9.582836181e-03f), f2pack(5.590641499e-02f, 5.590641499e-02f));
+    p = ffma2(p, r, f2pack(2.402409911e-01f, 2.402409911e-01f));
+    p = ffma2(p, r, f2pack(6.931241751e-01f, 6.931241751e-01f));
+  }
+  p = ffma2(p, r, f2pack(1.f, 1.f));
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// max over the row of s * c (c > 0: max(s) * c; c < 0: min(s) * c; c = 0: 0).
+__device__ __forceinline__ float row_max_scaled(const uint32_t (&sr)[BN], float c) {
+  float a[4];
+  if (c >= 0.f) {
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      a[g] = __uint_as_float(sr[32 * g]);
+#pragma unroll
+      for (int e = 1; e < 31; e += 2)
+        a[g] = max3f(a[g], __uint_as_float(sr[32 * g + e]), __uint_as_float(sr[32 * g + e + 1]));
+      a[g] = fmaxf(a[g], __uint_as_float(sr[32 * g + 31]));
+    }
+    return max3f(a[0], a[1], fmaxf(a[2], a[3])) * c;
+  }
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    a[g] = __uint_as_float(sr[32 * g]);
+#pragma unroll
+    for (int e = 1; e < 32; ++e) a[g] = fminf(a[g], __uint_as_float(sr[32 * g + e]));
+  }
+  return fminf(fminf(a[0], a[1]), fminf(a[2], a[3])) * c;
+}
+
+// P = 2^(s * cc + neg_m) for the row: EMU of every 4 pairs on the FMA pipe,
+// the rest on MUFU; packed to the input dtype and stored to TMEM columns
+// [taddr, taddr + 64) in two halves.  Returns the fp32 row sum; ymax gets the
+// largest fp32 weight (the one the rounding correction is taken from).
+template <bool BF16, int EMU>
+__device__ __forceinline__ float exp_store_row(const uint32_t (&sr)[BN], float cc, float neg_m, uint32_t taddr,
+                                               float& ymax) {
+  const uint64_t cc2 = f2pack(cc, cc), nm2 = f2pack(neg_m, neg_m);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+  float mx[2] = {0.f, 0.f};
+#pragma unroll
+  for (int h2 = 0; h2 < 2; ++h2) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int k = h2 * 64 + 2 * i;
+      const uint64_t x2 = ffma2(f2pack(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), cc2, nm2);
+      float y0, y1;
+      if ((i & 3) < EMU) {
+        exp2_poly_pair<BF16 ? 3 : 4>(x2, y0, y1);
+      } else {
+        float x0, x1;
+        f2unpack(x2, x0, x1);
+        y0 = ex2(x0);
+        y1 = ex2(x1);
+      }
+      acc[i & 3] = fadd2(acc[i & 3], f2pack(y0, y1));
+      mx[i & 1] = max3f(mx[i & 1], y0, y1);
+      pk[i] = pack2<BF16>(y0, y1);
+    }
+    tmem_st32(taddr + h2 * 32, pk);
+  }
+  ymax = fmaxf(mx[0], mx[1]);
+  float a0, a1;
+  f2unpack(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
+  return a0 + a1;
 }
 
 // ----------------------------------------------------------------------------- descriptors
@@ -424,48 +620,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr uint32_t IDESC_PV = idesc_f16(BM, D, FMT, 1);
 
   if (warp == LOAD_WARP) {
-    // ------------------------------------------------------------------ TMA producer
-    uint32_t kv_cnt = 0;
-    uint32_t q_use[NQ] = {0, 0};
-    bool ok = true;
-    for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
-      const Unit un = decode_unit(p, u);
-      const int n = max(un.n[0], un.n[1]);
-      for (int t = 0; t < NQ && ok; ++t) {
-        if (un.n[t] == 0) continue;
-        ok = wait_bar(bar(C::Q_EMPTY + t), (q_use[t] & 1u) ^ 1u, abort_flag, limit);
-        if (!ok) break;
-        ++q_use[t];
-        if (lane == 0) {
+    // ------------------------------------------------------------------ TMA producer (lane 0)
+    if (lane == 0) {
+      uint32_t kv_cnt = 0;
+      uint32_t q_use[NQ] = {0, 0};
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+        const Unit un = decode_unit(p, u);
+        const int n = max(un.n[0], un.n[1]);
+        for (int t = 0; t < NQ && ok; ++t) {
+          if (un.n[t] == 0) continue;
+          ok = wait_bar1(bar(C::Q_EMPTY + t), (q_use[t] & 1u) ^ 1u, abort_flag, limit);
+          if (!ok) break;
+          ++q_use[t];
           mbar_arrive_expect_tx(bar(C::Q_FULL + t), C::TILE_BYTES);
           const int s0 = un.r0 + t * BM;
           for (int bx = 0; bx < C::NBOX; ++bx)
             tma_load_4d(sQ + t * C::TILE_BYTES + bx * BOX_BYTES, &tmQ, bar(C::Q_FULL + t), bx * 64,
                         p.bhsd ? s0 : un.h, p.bhsd ? un.h : s0, un.b);
         }
-        __syncwarp();
-      }
-      for (int j = 0; j < n && ok; ++j) {
-        for (int kv = 0; kv < 2; ++kv) {
-          const uint32_t slot = kv_cnt % C::NSLOT;
-          const uint32_t use = kv_cnt / C::NSLOT;
-          ok = wait_bar(bar(C::KV_EMPTY + slot), (use & 1u) ^ 1u, abort_flag, limit);
-          if (!ok) break;
-          if (lane == 0) {
+        for (int j = 0; j < n && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const uint32_t slot = kv_cnt % C::NSLOT;
+            const uint32_t use = kv_cnt / C::NSLOT;
+            ok = wait_bar1(bar(C::KV_EMPTY + slot), (use & 1u) ^ 1u, abort_flag, limit);
+            if (!ok) break;
             mbar_arrive_expect_tx(bar(C::KV_FULL + slot), C::TILE_BYTES);
             const CUtensorMap* map = kv ? &tmV : &tmK;
             const int s0 = j * BN;
             for (int bx = 0; bx < C::NBOX; ++bx)
               tma_load_4d(sKV + slot * C::TILE_BYTES + bx * BOX_BYTES, map, bar(C::KV_FULL + slot),
                           bx * 64, p.bhsd ? s0 : un.h, p.bhsd ? un.h : s0, un.b);
+            ++kv_cnt;
           }
-          __syncwarp();
-          ++kv_cnt;
         }
       }
-    }
-    // Drain: wait until every load this warp issued has landed.
-    if (lane == 0) {
+      // Drain: wait until every load this thread issued has landed.
       const uint32_t first = kv_cnt > (uint32_t)C::NSLOT ? kv_cnt - C::NSLOT : 0u;
       for (uint32_t c = first; c < kv_cnt; ++c)
         drain_wait(bar(C::KV_FULL + c % C::NSLOT), (c / C::NSLOT) & 1u, limit);
@@ -475,11 +665,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------------ MMA issuer
+    // The whole warp runs this loop in step (warp-uniform waits and
+    // descriptors); each tcgen05 instruction is issued by one elected lane.
     uint32_t kv_cnt = 0;
     uint32_t q_use[NQ] = {0, 0}, p_use[NQ] = {0, 0}, o_use[NQ] = {0, 0};
     bool ok = true;
-    const uint32_t tS0 = tmem, tS1 = tmem + BM;
-    const uint32_t tO0 = tmem + 2 * BM, tO1 = tmem + 2 * BM + D;
+    // K-major SW128 descriptors of the Q tiles and of ring slot 0; a slot or a
+    // 16-element K step only moves the start address (16-byte units).
+    const uint64_t dQ0 = sdesc(sQ, 16, 1024);
+    const uint64_t dKV0 = sdesc(sKV, 16, 1024);
+    const uint64_t dV0 = sdesc(sKV, BOX_BYTES, 1024);
+    constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
+    auto qk = [&](int t, uint32_t kslot) {
+      const uint64_t a = dQ0 + (uint64_t)(t * TILE16);
+      const uint64_t b = dKV0 + (uint64_t)(kslot * TILE16);
+      const uint32_t d = tmem + t * BM;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
+        mma_ss_elect(d, a + off, b + off, IDESC_QK, kk > 0 ? 1u : 0u);
+      }
+    };
+    auto pv = [&](int t, uint32_t vslot, bool acc0) {
+      const uint64_t b = dV0 + (uint64_t)(vslot * TILE16);
+      const uint32_t d = tmem + 2 * BM + t * D, a = tmem + t * BM;
+#pragma unroll
+      for (int kk = 0; kk < BN / 16; ++kk)
+        mma_ts_elect(d, a + kk * 8, b + (uint64_t)(kk * 128), IDESC_PV, (acc0 || kk > 0) ? 1u : 0u);
+    };
     for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
       const Unit un = decode_unit(p, u);
       const int n = max(un.n[0], un.n[1]);
@@ -495,27 +708,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       ++kv_cnt;
       tc_fence_after();
-      if (lane == 0) {
-        for (int t = 0; t < NQ; ++t) {
-          if (un.n[t] == 0) continue;
-          const uint32_t qa = sQ + t * C::TILE_BYTES, ka = sKV + kslot * C::TILE_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
-            mma_ss(t ? tS1 : tS0, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), IDESC_QK,
-                   kk > 0);
-          }
-          tc_commit(bar(C::S_FULL + t));
-        }
-        tc_commit(bar(C::KV_EMPTY + kslot));
+      for (int t = 0; t < NQ; ++t) {
+        if (un.n[t] == 0) continue;
+        qk(t, kslot);
+        tc_commit_elect(bar(C::S_FULL + t));
       }
-      __syncwarp();
+      tc_commit_elect(bar(C::KV_EMPTY + kslot));
       for (int j = 0; j < n && ok; ++j) {
         const uint32_t vslot = kv_cnt % C::NSLOT;
         ok = wait_bar(bar(C::KV_FULL + vslot), (kv_cnt / C::NSLOT) & 1u, abort_flag, limit);
         if (!ok) break;
         ++kv_cnt;
-        const bool next_k = (j + 1 < n);
         bool k_ready = false;
         kslot = kv_cnt % C::NSLOT;
         for (int t = 0; t < NQ && ok; ++t) {
@@ -530,16 +733,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_fence_after();
           // O_t += P_t V_j   (P_t in TMEM, 16 keys = 8 packed columns per step)
-          if (lane == 0) {
-            const uint32_t va = sKV + vslot * C::TILE_BYTES;
-            const uint32_t tS = t ? tS1 : tS0;
-#pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk)
-              mma_ts(t ? tO1 : tO0, tS + kk * 8, sdesc(va + kk * 2048, BOX_BYTES, 1024), IDESC_PV,
-                     (j > 0 || kk > 0));
-            tc_commit(bar(C::O_FULL + t));
-          }
-          __syncwarp();
+          pv(t, vslot, j > 0);
+          if (j + 1 == un.n[t]) tc_commit_elect(bar(C::O_FULL + t));   // O_t final: the epilogue may read it
           if (j + 1 < un.n[t]) {
             if (!k_ready) {
               ok = wait_bar(bar(C::KV_FULL + kslot), (kv_cnt / C::NSLOT) & 1u, abort_flag, limit);
@@ -548,39 +743,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               k_ready = true;
               tc_fence_after();
             }
-            // S_t = Q_t K_{j+1}^T
-            if (lane == 0) {
-              const uint32_t qa = sQ + t * C::TILE_BYTES, ka = sKV + kslot * C::TILE_BYTES;
-#pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * BOX_BYTES + (kk & 3) * 32;
-                mma_ss(t ? tS1 : tS0, sdesc(qa + off, 16, 1024), sdesc(ka + off, 16, 1024), IDESC_QK,
-                       kk > 0);
-              }
-              tc_commit(bar(C::S_FULL + t));
-            }
-            __syncwarp();
+            // S_t = Q_t K_{j+1}^T; its commit also covers PV_t(j), so the
+            // softmax may rescale O_t once it has seen S_t(j+1).
+            qk(t, kslot);
+            tc_commit_elect(bar(C::S_FULL + t));
           }
         }
         if (!ok) break;
-        if (next_k && !k_ready) {  // cannot happen (n is the max over the tiles); keeps the ring in step
-          ok = wait_bar(bar(C::KV_FULL + kslot), (kv_cnt / C::NSLOT) & 1u, abort_flag, limit);
-          if (!ok) break;
-          ++kv_cnt;
-          k_ready = true;
-        }
-        if (lane == 0) {
-          tc_commit(bar(C::KV_EMPTY + vslot));
-          if (k_ready) tc_commit(bar(C::KV_EMPTY + kslot));
-        }
-        __syncwarp();
+        tc_commit_elect(bar(C::KV_EMPTY + vslot));
+        if (k_ready) tc_commit_elect(bar(C::KV_EMPTY + kslot));
       }
     }
-    // Drain: every MMA this thread issued has completed before TMEM is freed.
-    if (lane == 0) {
-      tc_commit(bar(C::DRAIN));
-      drain_wait(bar(C::DRAIN), 0, limit);
-    }
+    // Drain: every MMA this warp issued has completed before TMEM is freed.
+    tc_commit_elect(bar(C::DRAIN));
+    if (lane == 0) drain_wait(bar(C::DRAIN), 0, limit);
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ softmax warpgroups
@@ -591,7 +767,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tS = tmem + lane_bits + t * BM;
     const uint32_t tO = tmem + lane_bits + 2 * BM + t * D;
     const float c = p.scale_log2;
-    const bool c_neg = c < 0.f;
     uint32_t s_use = 0, o_use = 0, e_use = 0;
     bool ok = true;
     uint8_t* sQt = smem + C::SMEM_Q + t * C::TILE_BYTES;
@@ -603,113 +778,69 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int row = un.r0 + t * BM + rit;          // query row of this thread
       const int first_row = un.r0 + t * BM;
       float m = -INFINITY;                           // running max, log2 domain
-      float l = 0.f;                                 // running exp-sum
+      float l = 0.f;                                 // running exp-sum (for the LSE)
+      float ln = 0.f;                                // l with each tile's top weight as rounded in P (for O)
       float m_use = 0.f;
       for (int j = 0; j < nt; ++j) {
+        // S_t(j) is complete; its commit also covers P_t(j-1) V(j-1), so O_t is settled.
         ok = wait_bar(bar(C::S_FULL + t), s_use & 1u, abort_flag, limit);
         if (!ok) break;
         ++s_use;
         tc_fence_after();
-        float s[BN];
-        {
-          uint32_t r[32];
-#pragma unroll
-          for (int q4 = 0; q4 < BN / 32; ++q4) {
-            tmem_ld32(tS + q4 * 32, r);
-            tmem_wait_ld();
-            reg_fence(r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s[q4 * 32 + i] = __uint_as_float(r[i]);
-          }
-        }
+        uint32_t sr[BN];                               // this row of S_t (fp32 bits)
+        tmem_ld_cols<BN / 32>(tS, sr);
         const int c0 = j * BN;
-        const bool tail = (c0 + BN > p.Sk);
-        const bool diag = p.causal && (c0 + BN - 1 > first_row);
-        float cc = c;
+        const bool masked = (c0 + BN > p.Sk) || (p.causal && (c0 + BN - 1 > first_row));
         float m_blk;
-        if (tail || diag) {
-          // masked tile: work on scaled logits, masked entries -> -inf
+        if (masked) {
+          // diagonal or ragged tile: scaled logits, masked entries -> -inf
           int lim = p.Sk - 1 - c0;
           if (p.causal) lim = min(lim, row - c0);
           float mx = -INFINITY;
 #pragma unroll
           for (int k = 0; k < BN; ++k) {
-            const float tv = (k > lim) ? -INFINITY : s[k] * c;
-            s[k] = tv;
+            const float tv = (k > lim) ? -INFINITY : __uint_as_float(sr[k]) * c;
+            sr[k] = __float_as_uint(tv);
             mx = fmaxf(mx, tv);
           }
           m_blk = mx;
-          cc = 1.f;
-        } else if (!c_neg) {
-          float a0 = s[0], a1 = s[1], a2 = s[2], a3 = s[3];
-#pragma unroll
-          for (int k = 4; k < BN; k += 4) {
-            a0 = fmaxf(a0, s[k]);
-            a1 = fmaxf(a1, s[k + 1]);
-            a2 = fmaxf(a2, s[k + 2]);
-            a3 = fmaxf(a3, s[k + 3]);
-          }
-          m_blk = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * c;
         } else {
-          float a0 = s[0], a1 = s[1], a2 = s[2], a3 = s[3];
-#pragma unroll
-          for (int k = 4; k < BN; k += 4) {
-            a0 = fminf(a0, s[k]);
-            a1 = fminf(a1, s[k + 1]);
-            a2 = fminf(a2, s[k + 2]);
-            a3 = fminf(a3, s[k + 3]);
-          }
-          m_blk = fminf(fminf(a0, a1), fminf(a2, a3)) * c;
+          m_blk = row_max_scaled(sr, c);
         }
-        const float m_new = fmaxf(m, m_blk);
-        m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = ex2(m - m_use);          // 0 on the first tile, 1 if m did not grow
-        m = m_new;
-        const float neg_m = -m_use;
-        float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
-        uint32_t pk[BN / 2];
+        // The running max moves only when the tile's max exceeds it by more
+        // than RESCALE_LOG2; otherwise P may reach 2^RESCALE_LOG2 and O, l keep
+        // their scale (the result is the same: O and l share the reference m).
+        const float m_cand = fmaxf(m, m_blk);
+        const bool grow = m_cand > m + RESCALE_LOG2;
+        const float m_prev = m;
+        if (grow) m = m_cand;
+        m_use = (m == -INFINITY) ? 0.f : m;
+        const float alpha = grow ? ex2(m_prev - m_use) : 1.f;   // 0 when m_prev = -inf
+        // P = 2^(s * c - m) written to TMEM (first 64 columns of S_t), row sum in fp32
+        float p_top;
+        const float rowsum = masked ? exp_store_row<BF16, 0>(sr, 1.f, -m_use, tS, p_top)
+                                    : exp_store_row<BF16, EMU_PAIRS>(sr, c, -m_use, tS, p_top);
+        // P enters P.V rounded to the input dtype.  The largest weight of the
+        // tile can exceed 1 (stale max), where rounding is not exact; adding its
+        // rounding error to the normaliser makes O divide by the same value it
+        // multiplied by, so a dominant key carries no extra error.
+        const float corr = round_to_input<BF16>(p_top) - p_top;
+        l = l * alpha + rowsum;
+        ln = ln * alpha + rowsum + corr;
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          uint32_t orow[D];
+          tmem_ld_cols<D / 32>(tO, orow);
+          const uint64_t a2 = f2pack(alpha, alpha);
 #pragma unroll
-        for (int k = 0; k < BN; k += 4) {
-          const float p0 = ex2(fmaf(s[k], cc, neg_m));
-          const float p1 = ex2(fmaf(s[k + 1], cc, neg_m));
-          const float p2 = ex2(fmaf(s[k + 2], cc, neg_m));
-          const float p3 = ex2(fmaf(s[k + 3], cc, neg_m));
-          rs0 += p0;
-          rs1 += p1;
-          rs2 += p2;
-          rs3 += p3;
-          pk[k / 2] = pack2<BF16>(p0, p1);
-          pk[k / 2 + 1] = pack2<BF16>(p2, p3);
-        }
-        l = l * alpha + ((rs0 + rs1) + (rs2 + rs3));
-        // P_t -> TMEM (first 64 columns of S_t)
-        {
-          uint32_t r[32];
-#pragma unroll
-          for (int h2 = 0; h2 < BN / 64; ++h2) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = pk[h2 * 32 + i];
-            tmem_st32(tS + h2 * 32, r);
+          for (int i = 0; i < D / 2; ++i) {
+            float o0, o1;
+            f2unpack(fmul2(f2pack(__uint_as_float(orow[2 * i]), __uint_as_float(orow[2 * i + 1])), a2), o0, o1);
+            orow[2 * i] = __float_as_uint(o0);
+            orow[2 * i + 1] = __float_as_uint(o1);
           }
-        }
-        if (j > 0) {
-          // O_t of the previous tile is complete; rescale it if any row's max grew
-          ok = wait_bar(bar(C::O_FULL + t), o_use & 1u, abort_flag, limit);
-          if (!ok) break;
-          ++o_use;
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
-            uint32_t r[32];
 #pragma unroll
-            for (int q4 = 0; q4 < D / 32; ++q4) {
-              tmem_ld32(tO + q4 * 32, r);
-              tmem_wait_ld();
-              reg_fence(r);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-              tmem_st32(tO + q4 * 32, r);
-            }
-          }
+          for (int q4 = 0; q4 < D / 32; ++q4)
+            tmem_st32(tO + q4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&orow[32 * q4]));
         }
         tmem_wait_st();
         tc_fence_before();
@@ -722,7 +853,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       ++o_use;
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = 1.f / ln;
       {
         uint32_t r[32];
 #pragma unroll
