@@ -60,15 +60,23 @@ constexpr int BM = 128;             // query rows per tile (one TMEM lane per ro
 constexpr int BN = 128;             // keys per K / V tile
 constexpr int NQ = 2;               // query tiles per work unit (ping-pong)
 constexpr int UNIT_ROWS = NQ * BM;  // 256
-constexpr int NUM_THREADS = 320;    // warps 0-7 softmax, 8 load, 9 MMA
+constexpr int NUM_THREADS = 384;    // warps 0-7 softmax, 8 load, 9 MMA, 10-11 idle (producer warpgroup)
+// Register split (setmaxnreg): the launch gives 384 x 168 = 64512 registers;
+// the producer warpgroup drops to 112 per thread and the two softmax
+// warpgroups rise to 184: 128 x 112 + 256 x 184 = 61440, within the launch.
+constexpr int REGS_PRODUCER = 112;
+constexpr int REGS_SOFTMAX = 184;
+static_assert(128 * REGS_PRODUCER + 256 * REGS_SOFTMAX <= NUM_THREADS * 168, "register split exceeds the launch");
 constexpr int LOAD_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr int TMEM_COLS = 512;
 constexpr int BOX_BYTES = BM * 128;  // one 128-row x 64-element (128-byte) TMA box
 #ifndef FA_RESCALE_LOG2
-#define FA_RESCALE_LOG2 8.0f
+#define FA_RESCALE_LOG2 15.0f
 #endif
 constexpr float RESCALE_LOG2 = FA_RESCALE_LOG2;  // O / l are rescaled only when a row max grows by more (log2 units)
+constexpr float RESCALE_POW2 = (float)(1u << (int)FA_RESCALE_LOG2);  // 2^RESCALE_LOG2
+constexpr float HEADROOM_LOG2 = 8.0f;  // bf16 only: a moved reference sits this far above the tile max
 #ifndef FA_EMU_PAIRS
 #define FA_EMU_PAIRS 1
 #endif
@@ -422,14 +430,16 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 // 1.5 * 2^23 - (x + 1.5 * 2^23) = -j exactly and r = x - j lies in [-1/2, 1/2].
 // 2^r is a polynomial (constant term 1; near-minimax in relative error, fitted
 // by csrc/gen_exp2_poly.py: 1.0e-4 at degree 3, 2.9e-6 at degree 4), and 2^j
-// is added to its exponent field.  x is clamped at -125 so the exponent stays
-// normal; 2^-125 stands in for anything smaller.
+// is added to its exponent field.  x is clamped to [-125, 64] so the exponent
+// stays normal: 2^-125 stands in for anything smaller, and an argument above
+// 64 (only possible on a rejected speculative pass, see the softmax) still
+// gives a large positive value.
 template <int DEG>
 __device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& y0, float& y1) {
   float x0, x1;
   f2unpack(x2, x0, x1);
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
+  x0 = fminf(fmaxf(x0, -125.f), 64.f);
+  x1 = fminf(fmaxf(x1, -125.f), 64.f);
   const uint64_t magic = f2pack(12582912.f, 12582912.f);
   const uint64_t t = fadd2(f2pack(x0, x1), magic);
   const uint64_t neg_j = ffma2(t, f2pack(-1.f, -1.f), magic);
@@ -475,38 +485,32 @@ __device__ __forceinline__ float row_max_scaled(const uint32_t (&sr)[BN], float 
 }
 
 // P = 2^(s * cc + neg_m) for the row: EMU of every 4 pairs on the FMA pipe,
-// the rest on MUFU; packed to the input dtype and stored to TMEM columns
-// [taddr, taddr + 64) in two halves.  Returns the fp32 row sum; ymax gets the
-// largest fp32 weight (the one the rounding correction is taken from).
+// the rest on MUFU; packed to the input dtype into pk (two per 32-bit word).
+// Returns the fp32 row sum; ymax gets the largest fp32 weight (the one the
+// rounding correction is taken from, and the speculation check).
 template <bool BF16, int EMU>
-__device__ __forceinline__ float exp_store_row(const uint32_t (&sr)[BN], float cc, float neg_m, uint32_t taddr,
-                                               float& ymax) {
+__device__ __forceinline__ float exp_pack_row(const uint32_t (&sr)[BN], float cc, float neg_m, uint32_t (&pk)[BN / 2],
+                                              float& ymax) {
   const uint64_t cc2 = f2pack(cc, cc), nm2 = f2pack(neg_m, neg_m);
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-  float mx[2] = {0.f, 0.f};
+  float mx[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int h2 = 0; h2 < 2; ++h2) {
-    uint32_t pk[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int k = h2 * 64 + 2 * i;
-      const uint64_t x2 = ffma2(f2pack(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), cc2, nm2);
-      float y0, y1;
-      if ((i & 3) < EMU) {
-        exp2_poly_pair<BF16 ? 3 : 4>(x2, y0, y1);
-      } else {
-        float x0, x1;
-        f2unpack(x2, x0, x1);
-        y0 = ex2(x0);
-        y1 = ex2(x1);
-      }
-      acc[i & 3] = fadd2(acc[i & 3], f2pack(y0, y1));
-      mx[i & 1] = max3f(mx[i & 1], y0, y1);
-      pk[i] = pack2<BF16>(y0, y1);
+  for (int i = 0; i < BN / 2; ++i) {
+    const uint64_t x2 = ffma2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), cc2, nm2);
+    float y0, y1;
+    if ((i & 3) < EMU) {
+      exp2_poly_pair<BF16 ? 3 : 4>(x2, y0, y1);
+    } else {
+      float x0, x1;
+      f2unpack(x2, x0, x1);
+      y0 = ex2(x0);
+      y1 = ex2(x1);
     }
-    tmem_st32(taddr + h2 * 32, pk);
+    acc[i & 3] = fadd2(acc[i & 3], f2pack(y0, y1));
+    mx[i & 7] = max3f(mx[i & 7], y0, y1);
+    pk[i] = pack2<BF16>(y0, y1);
   }
-  ymax = fmaxf(mx[0], mx[1]);
+  ymax = max3f(max3f(mx[0], mx[1], mx[2]), max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
   float a0, a1;
   f2unpack(fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3])), a0, a1);
   return a0 + a1;
@@ -619,7 +623,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr uint32_t IDESC_QK = idesc_f16(BM, BN, FMT, 0);
   constexpr uint32_t IDESC_PV = idesc_f16(BM, D, FMT, 1);
 
-  if (warp == LOAD_WARP) {
+  if (warp >= LOAD_WARP) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
+   if (warp == LOAD_WARP) {
     // ------------------------------------------------------------------ TMA producer (lane 0)
     if (lane == 0) {
       uint32_t kv_cnt = 0;
@@ -628,8 +634,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
         const Unit un = decode_unit(p, u);
         const int n = max(un.n[0], un.n[1]);
-        for (int t = 0; t < NQ && ok; ++t) {
-          if (un.n[t] == 0) continue;
+#pragma unroll
+        for (int t = 0; t < NQ; ++t) {
+          if (un.n[t] == 0 || !ok) continue;
           ok = wait_bar1(bar(C::Q_EMPTY + t), (q_use[t] & 1u) ^ 1u, abort_flag, limit);
           if (!ok) break;
           ++q_use[t];
@@ -659,6 +666,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t first = kv_cnt > (uint32_t)C::NSLOT ? kv_cnt - C::NSLOT : 0u;
       for (uint32_t c = first; c < kv_cnt; ++c)
         drain_wait(bar(C::KV_FULL + c % C::NSLOT), (c / C::NSLOT) & 1u, limit);
+#pragma unroll
       for (int t = 0; t < NQ; ++t)
         if (q_use[t]) drain_wait(bar(C::Q_FULL + t), (q_use[t] - 1) & 1u, limit);
     }
@@ -696,8 +704,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
       const Unit un = decode_unit(p, u);
       const int n = max(un.n[0], un.n[1]);
-      for (int t = 0; t < NQ && ok; ++t) {
-        if (un.n[t] == 0) continue;
+#pragma unroll
+      for (int t = 0; t < NQ; ++t) {
+        if (un.n[t] == 0 || !ok) continue;
         ok = wait_bar(bar(C::Q_FULL + t), q_use[t] & 1u, abort_flag, limit);
         ++q_use[t];
       }
@@ -708,6 +717,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       ++kv_cnt;
       tc_fence_after();
+#pragma unroll
       for (int t = 0; t < NQ; ++t) {
         if (un.n[t] == 0) continue;
         qk(t, kslot);
@@ -721,8 +731,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++kv_cnt;
         bool k_ready = false;
         kslot = kv_cnt % C::NSLOT;
-        for (int t = 0; t < NQ && ok; ++t) {
-          if (j >= un.n[t]) continue;
+#pragma unroll
+        for (int t = 0; t < NQ; ++t) {
+          if (j >= un.n[t] || !ok) continue;
           ok = wait_bar(bar(C::P_FULL + t), p_use[t] & 1u, abort_flag, limit);
           if (!ok) break;
           ++p_use[t];
@@ -758,7 +769,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_commit_elect(bar(C::DRAIN));
     if (lane == 0) drain_wait(bar(C::DRAIN), 0, limit);
     __syncwarp();
+   }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
     // ------------------------------------------------------------------ softmax warpgroups
     const int t = warp >> 2;               // query tile of this warpgroup
     const int quad = warp & 3;             // TMEM lane quadrant
@@ -773,7 +786,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
       const Unit un = decode_unit(p, u);
-      const int nt = un.n[t];
+      const int nt = t ? un.n[1] : un.n[0];
       if (nt == 0) continue;
       const int row = un.r0 + t * BM + rit;          // query row of this thread
       const int first_row = un.r0 + t * BM;
@@ -787,39 +800,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!ok) break;
         ++s_use;
         tc_fence_after();
-        uint32_t sr[BN];                               // this row of S_t (fp32 bits)
-        tmem_ld_cols<BN / 32>(tS, sr);
         const int c0 = j * BN;
         const bool masked = (c0 + BN > p.Sk) || (p.causal && (c0 + BN - 1 > first_row));
-        float m_blk;
-        if (masked) {
-          // diagonal or ragged tile: scaled logits, masked entries -> -inf
-          int lim = p.Sk - 1 - c0;
-          if (p.causal) lim = min(lim, row - c0);
-          float mx = -INFINITY;
+        const float cc = masked ? 1.f : c;
+        int lim = p.Sk - 1 - c0;
+        if (p.causal) lim = min(lim, row - c0);
+        // this row of S_t from TMEM; diagonal / ragged tiles become scaled logits
+        // with masked entries at -inf
+        auto load_s = [&](uint32_t (&sr)[BN]) {
+          tmem_ld_cols<BN / 32>(tS, sr);
+          if (masked) {
 #pragma unroll
-          for (int k = 0; k < BN; ++k) {
-            const float tv = (k > lim) ? -INFINITY : __uint_as_float(sr[k]) * c;
-            sr[k] = __float_as_uint(tv);
-            mx = fmaxf(mx, tv);
+            for (int k = 0; k < BN; ++k)
+              sr[k] = __float_as_uint((k > lim) ? -INFINITY : __uint_as_float(sr[k]) * c);
           }
-          m_blk = mx;
-        } else {
-          m_blk = row_max_scaled(sr, c);
-        }
-        // The running max moves only when the tile's max exceeds it by more
-        // than RESCALE_LOG2; otherwise P may reach 2^RESCALE_LOG2 and O, l keep
-        // their scale (the result is the same: O and l share the reference m).
-        const float m_cand = fmaxf(m, m_blk);
-        const bool grow = m_cand > m + RESCALE_LOG2;
+        };
+        uint32_t sr[BN];
+        uint32_t pk[BN / 2];
+        load_s(sr);
+        // P = 2^(s * cc - m), packed in registers; written to TMEM (the first
+        // 64 columns of S_t) only once accepted.  From the second tile on, the
+        // exponentials are taken against the current reference m straight
+        // away: the reference must move only if this tile's max exceeds it by
+        // more than RESCALE_LOG2, which shows as a weight above
+        // 2^RESCALE_LOG2.  Then (rarely) the warp reloads S (still intact in
+        // TMEM), takes the exact tile max, moves m and recomputes P.  The first
+        // tile of a unit starts from the exact max.
+        float p_top = 0.f, rowsum = 0.f;
+        bool grow = false;
         const float m_prev = m;
-        if (grow) m = m_cand;
-        m_use = (m == -INFINITY) ? 0.f : m;
+        bool exact = (j == 0);
+        if (!exact) {
+          rowsum = masked ? exp_pack_row<BF16, 0>(sr, cc, -m_use, pk, p_top)
+                          : exp_pack_row<BF16, EMU_PAIRS>(sr, cc, -m_use, pk, p_top);
+          exact = __any_sync(0xffffffffu, !(p_top <= RESCALE_POW2));
+          if (exact) load_s(sr);
+        }
+        if (exact) {
+          const float m_blk = row_max_scaled(sr, cc);
+          const float m_cand = fmaxf(m, m_blk);
+          grow = (m == -INFINITY) || (m_cand > m + RESCALE_LOG2) || !(p_top <= RESCALE_POW2);
+          // bf16 keeps the fp32 exponent range, so the new reference is set
+          // above the max (weights <= 2^-HEADROOM) and later tiles may grow by
+          // HEADROOM + RESCALE_LOG2 before the next move; fp16 keeps the max.
+          if (grow) m = m_cand + (BF16 ? HEADROOM_LOG2 : 0.f);
+          m_use = (m == -INFINITY) ? 0.f : m;
+          rowsum = masked ? exp_pack_row<BF16, 0>(sr, cc, -m_use, pk, p_top)
+                          : exp_pack_row<BF16, EMU_PAIRS>(sr, cc, -m_use, pk, p_top);
+        }
+#pragma unroll
+        for (int h2 = 0; h2 < BN / 64; ++h2)
+          tmem_st32(tS + h2 * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32 * h2]));
         const float alpha = grow ? ex2(m_prev - m_use) : 1.f;   // 0 when m_prev = -inf
-        // P = 2^(s * c - m) written to TMEM (first 64 columns of S_t), row sum in fp32
-        float p_top;
-        const float rowsum = masked ? exp_store_row<BF16, 0>(sr, 1.f, -m_use, tS, p_top)
-                                    : exp_store_row<BF16, EMU_PAIRS>(sr, c, -m_use, tS, p_top);
         // P enters P.V rounded to the input dtype.  The largest weight of the
         // tile can exceed 1 (stale max), where rounding is not exact; adding its
         // rounding error to the normaliser makes O divide by the same value it
