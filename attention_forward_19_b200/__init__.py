@@ -36,8 +36,8 @@ FA_BF16 = 1
 LAYOUTS = {"BSND": FA_BSND, "BHSD": FA_BHSD}
 
 # Names every public symbol of include/fa_fwd.h.
-EXPORTED_SYMBOLS = ("fa_fwd", "fa_device_status", "fa_query_support", "fa_status_string",
-                    "fa_last_cuda_error", "fa_version")
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_device_status", "fa_query_support",
+                    "fa_status_string", "fa_last_cuda_error", "fa_version")
 
 
 class FaError(RuntimeError):
@@ -74,6 +74,11 @@ def load_library(path=None, rebuild_if_stale=True):
     i64, vp, c_int, c_float = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.fa_fwd.restype = c_int
     lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, vp]
+    lib.fa_fwd_ws.restype = c_int
+    lib.fa_fwd_ws.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, vp,
+                              ctypes.c_size_t, vp]
+    lib.fa_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.fa_fwd_workspace_size.argtypes = []
     lib.fa_device_status.restype = c_int
     lib.fa_device_status.argtypes = [vp]
     lib.fa_query_support.restype = c_int
@@ -96,6 +101,18 @@ def fa_fwd(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, strea
     lib = load_library()
     return lib.fa_fwd(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
                       int(bool(causal)), float(scale), int(dtype), stream)
+
+
+def fa_fwd_ws(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, workspace, workspace_bytes,
+              stream):
+    """The C fa_fwd_ws (dynamic schedule) with raw pointers and sizes; returns the fa_status code."""
+    lib = load_library()
+    return lib.fa_fwd_ws(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
+                         int(bool(causal)), float(scale), int(dtype), workspace, int(workspace_bytes), stream)
+
+
+def fa_fwd_workspace_size():
+    return load_library().fa_fwd_workspace_size()
 
 
 def fa_device_status(stream=None):
@@ -148,13 +165,16 @@ def _dims(q, k, layout, head_num=None):
 
 
 def flash_attention_forward(q, k, v, layout="BSND", causal=False, scale=None, head_num=None,
-                            out=None, lse=None, stream=None):
+                            out=None, lse=None, stream=None, schedule="dynamic", workspace=None):
     """Attention forward on CUDA tensors through the C ABI.
 
     q: [B, Sq, H, D] (BSND) or [B, H, Sq, D] (BHSD); k, v likewise with Sk.
     scale=None uses 1/sqrt(D).  Returns (o, lse): o like q, lse fp32 [B, H, Sq].
     out / lse may be given to reuse buffers.  Runs on `stream` (default: the
     current torch stream) without synchronising.
+    schedule="dynamic" calls fa_fwd_ws (work units handed out from a counter
+    in `workspace`, a uint8 CUDA tensor of fa_fwd_workspace_size() bytes,
+    allocated here when not given); "static" calls fa_fwd (no workspace).
     """
     import torch
     lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
@@ -180,10 +200,24 @@ def flash_attention_forward(q, k, v, layout="BSND", causal=False, scale=None, he
     if stream is None:
         stream = torch.cuda.current_stream(q.device) if q.is_cuda else None
     sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
-    st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                B, H, Sq, Sk, D, lay, causal, scale, dt, sptr)
+    if schedule == "static":
+        st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                    B, H, Sq, Sk, D, lay, causal, scale, dt, sptr)
+        where = "fa_fwd"
+    elif schedule == "dynamic":
+        nbytes = fa_fwd_workspace_size()
+        if workspace is None:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+        if workspace.numel() * workspace.element_size() < nbytes or not workspace.is_contiguous():
+            raise ValueError(f"workspace must be a contiguous tensor of at least {nbytes} bytes")
+        st = fa_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                       B, H, Sq, Sk, D, lay, causal, scale, dt, workspace.data_ptr(),
+                       workspace.numel() * workspace.element_size(), sptr)
+        where = "fa_fwd_ws"
+    else:
+        raise ValueError(f"schedule must be 'dynamic' or 'static', not {schedule!r}")
     if st != FA_OK:
-        raise FaError(st, "fa_fwd")
+        raise FaError(st, where)
     return out, lse
 
 

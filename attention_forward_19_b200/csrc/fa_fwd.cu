@@ -71,6 +71,8 @@ constexpr int LOAD_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr int TMEM_COLS = 512;
 constexpr int BOX_BYTES = BM * 128;  // one 128-row x 64-element (128-byte) TMA box
+constexpr int UQ_DEPTH = 4;           // unit ids in flight between the producer and the consumers
+constexpr int UQ_CONSUMERS = 9;       // arrivals that free a unit-id slot: the MMA warp + 8 softmax warps
 #ifndef FA_RESCALE_LOG2
 #define FA_RESCALE_LOG2 15.0f
 #endif
@@ -98,16 +100,19 @@ struct Cfg {
   static constexpr int O_EMPTY = O_FULL + NQ;
   static constexpr int EPI = O_EMPTY + NQ;
   static constexpr int DRAIN = EPI + NQ;
-  static constexpr int NBAR = DRAIN + 1;
+  static constexpr int UQ_FULL = DRAIN + 1;     // unit-id ring: producer -> MMA warp and softmax warps
+  static constexpr int UQ_EMPTY = UQ_FULL + UQ_DEPTH;
+  static constexpr int NBAR = UQ_EMPTY + UQ_DEPTH;
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_KV = NQ * TILE_BYTES;
   static constexpr int SMEM_BAR = SMEM_KV + NSLOT * TILE_BYTES;
-  static constexpr int SMEM_MISC = SMEM_BAR + NBAR * 8;       // tmem address, abort flag
-  static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;    // + slack for 1024-byte alignment
+  static constexpr int SMEM_MISC = SMEM_BAR + NBAR * 8;       // tmem address, abort flag, unit-id ring
+  static constexpr int SMEM_BYTES = SMEM_MISC + 8 + 4 * UQ_DEPTH + 1024;  // + slack for 1024-byte alignment
 };
 
 struct Params {
   float* lse;
+  unsigned int* sched;  // work counter for the dynamic schedule (zeroed before launch), or nullptr: static
   int B, H, Sq, Sk;
   int nqb;             // query units per head: ceil(Sq / 256)
   int tk;              // key tiles: ceil(Sk / 128)
@@ -586,6 +591,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t bars = smem_u32(smem + C::SMEM_BAR);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 4);
+  volatile int* uq_ids = reinterpret_cast<volatile int*>(smem + C::SMEM_MISC + 8);
   auto bar = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
 
   const int warp = threadIdx.x >> 5;
@@ -607,6 +613,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar(C::EPI + t), BM);
     }
     mbar_init(bar(C::DRAIN), 1);
+    for (int i = 0; i < UQ_DEPTH; ++i) {
+      mbar_init(bar(C::UQ_FULL + i), 1);
+      mbar_init(bar(C::UQ_EMPTY + i), UQ_CONSUMERS);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -631,7 +641,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t kv_cnt = 0;
       uint32_t q_use[NQ] = {0, 0};
       bool ok = true;
-      for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+      // Work units: the first is blockIdx.x; later ones come from the work
+      // counter (dynamic schedule: units handed out in longest-first order)
+      // or every gridDim.x-th unit (static schedule).  Each id, and finally an
+      // end-of-work id, is passed to the MMA warp and the softmax warps
+      // through the unit-id ring.
+      int u = blockIdx.x;
+      uint32_t uq_pos = 0;
+      while (ok) {
+        const uint32_t qs = uq_pos % UQ_DEPTH;
+        ok = wait_bar1(bar(C::UQ_EMPTY + qs), ((uq_pos / UQ_DEPTH) & 1u) ^ 1u, abort_flag, limit);
+        if (!ok) break;
+        uq_ids[qs] = u;
+        mbar_arrive(bar(C::UQ_FULL + qs));
+        ++uq_pos;
+        if (u >= p.total_units) break;
         const Unit un = decode_unit(p, u);
         const int n = max(un.n[0], un.n[1]);
 #pragma unroll
@@ -661,6 +685,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ++kv_cnt;
           }
         }
+        // The next unit is claimed only now, once every load of this one is
+        // issued: the CTA then gets work about when it can start on it, which
+        // keeps the longest-first hand-out balanced.
+        u = p.sched ? (int)(gridDim.x + atomicAdd(p.sched, 1u)) : u + (int)gridDim.x;
       }
       // Drain: wait until every load this thread issued has landed.
       const uint32_t first = kv_cnt > (uint32_t)C::NSLOT ? kv_cnt - C::NSLOT : 0u;
@@ -701,7 +729,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int kk = 0; kk < BN / 16; ++kk)
         mma_ts_elect(d, a + kk * 8, b + (uint64_t)(kk * 128), IDESC_PV, (acc0 || kk > 0) ? 1u : 0u);
     };
-    for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+    uint32_t uq_pos = 0;
+    while (ok) {
+      const uint32_t qs = uq_pos % UQ_DEPTH;
+      ok = wait_bar(bar(C::UQ_FULL + qs), (uq_pos / UQ_DEPTH) & 1u, abort_flag, limit);
+      if (!ok) break;
+      const int u = uq_ids[qs];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::UQ_EMPTY + qs));
+      ++uq_pos;
+      if (u >= p.total_units) break;
       const Unit un = decode_unit(p, u);
       const int n = max(un.n[0], un.n[1]);
 #pragma unroll
@@ -784,7 +821,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     uint8_t* sQt = smem + C::SMEM_Q + t * C::TILE_BYTES;
 
-    for (int u = blockIdx.x; u < p.total_units && ok; u += gridDim.x) {
+    uint32_t uq_pos = 0;
+    while (ok) {
+      const uint32_t qs = uq_pos % UQ_DEPTH;
+      ok = wait_bar(bar(C::UQ_FULL + qs), (uq_pos / UQ_DEPTH) & 1u, abort_flag, limit);
+      if (!ok) break;
+      const int u = uq_ids[qs];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::UQ_EMPTY + qs));
+      ++uq_pos;
+      if (u >= p.total_units) break;
       const Unit un = decode_unit(p, u);
       const int nt = t ? un.n[1] : un.n[0];
       if (nt == 0) continue;
@@ -1046,13 +1092,14 @@ constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
-}  // namespace
+constexpr size_t kWorkspaceBytes = 16;  // the work counter of the dynamic schedule (4 bytes used)
 
-extern "C" {
-
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
-                 int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
-                 void* stream) {
+// Validates the arguments, builds the tensor maps and launches the kernel.
+// sched: the dynamic-schedule counter in device memory (zeroed here, on the
+// stream, before the launch), or nullptr for the static schedule.
+fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                   int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
+                   unsigned int* sched, void* stream) {
   // ---- arguments that need no device
   if (B <= 0 || H <= 0 || Sq < 0 || Sk <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
   if (layout != FA_BSND && layout != FA_BHSD) return FA_ERR_INVALID_ARG;
@@ -1082,8 +1129,9 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail((int)e);
   if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
-  const void* ptrs[5] = {q, k, v, o, lse};
+  const void* ptrs[6] = {q, k, v, o, lse, sched};
   for (const void* ptr : ptrs) {
+    if (!ptr) continue;   // only sched may be null here
     fa_status st = check_device_ptr(ptr, dev);
     if (st != FA_OK) return st;
   }
@@ -1127,6 +1175,11 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 
   const int grid = (int)(prm.total_units < sms ? prm.total_units : sms);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  prm.sched = sched;
+  if (sched) {
+    e = cudaMemsetAsync(sched, 0, sizeof(unsigned int), s);
+    if (e != cudaSuccess) return cuda_fail((int)e);
+  }
   bool* cfg = g_dev[dev].configured;
   if (D == 128)
     return dtype == FA_BF16 ? launch<128, true>(prm, mq, mk, mv, mo, grid, &cfg[0], s)
@@ -1134,6 +1187,40 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   return dtype == FA_BF16 ? launch<64, true>(prm, mq, mk, mv, mo, grid, &cfg[2], s)
                           : launch<64, false>(prm, mq, mk, mv, mo, grid, &cfg[3], s);
 }
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                 int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
+                 void* stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, nullptr, stream);
+}
+
+fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                    int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace) {
+    // the sizes may still make the call a no-op; otherwise a workspace is required
+    if (Sq == 0 && B > 0 && H > 0 && Sk > 0) return FA_OK;
+    return FA_ERR_INVALID_ARG;
+  }
+  if (workspace_bytes < kWorkspaceBytes) return FA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) & 15u) return FA_ERR_MISALIGNED;
+  if (B > 0 && H > 0 && D > 0 && Sq > 0 && Sk > 0) {
+    const size_t qbytes = (size_t)(B * H * Sq * D) * 2, kvbytes = (size_t)(B * H * Sk * D) * 2;
+    const size_t lbytes = (size_t)(B * H * Sq) * 4;
+    if ((q && overlaps(workspace, workspace_bytes, q, qbytes)) || (k && overlaps(workspace, workspace_bytes, k, kvbytes)) ||
+        (v && overlaps(workspace, workspace_bytes, v, kvbytes)) || (o && overlaps(workspace, workspace_bytes, o, qbytes)) ||
+        (lse && overlaps(workspace, workspace_bytes, lse, lbytes)))
+      return FA_ERR_ALIAS;
+  }
+  return fwd_impl(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype,
+                  static_cast<unsigned int*>(workspace), stream);
+}
+
+size_t fa_fwd_workspace_size(void) { return kWorkspaceBytes; }
 
 fa_status fa_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

@@ -192,11 +192,13 @@ def run_native(args, rank, world, local_rank):
     q, k, v = make_qkv(w, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
+    # work counter of the dynamic schedule (fa_fwd_ws); zeroed by the library before every launch
+    ws = torch.empty(fa.fa_fwd_workspace_size(), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
         fa.flash_attention_forward(q, k, v, layout=w.layout, causal=w.causal, scale=w.scale, out=o, lse=lse,
-                                   stream=stream)
+                                   stream=stream, schedule="dynamic", workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -243,7 +245,7 @@ def run_native(args, rank, world, local_rank):
         dk = hk.to(dev, non_blocking=True)
         dv = hv.to(dev, non_blocking=True)
         do, dl = fa.flash_attention_forward(dq, dk, dv, layout=w.layout, causal=w.causal, scale=w.scale,
-                                            stream=stream)
+                                            stream=stream, schedule="dynamic", workspace=ws)
         ho.copy_(do, non_blocking=True)
         hl.copy_(dl, non_blocking=True)
 
@@ -304,7 +306,8 @@ def run_native(args, rank, world, local_rank):
                 "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
         "gpu_launches": args.steps,
         "clocks": clk,
-        "kernel": "fa::fa_fwd_kernel<128, true> (libfa_fwd.so)",
+        "kernel": "fa::fa_fwd_kernel<128, true> via fa_fwd_ws (dynamic schedule; libfa_fwd.so)",
+        "gpu_launches_note": "one fa_fwd_kernel launch per step (plus the library's 4-byte cudaMemsetAsync of the work counter)",
     }
     return line
 

@@ -43,6 +43,7 @@
 #ifndef FA_FWD_H
 #define FA_FWD_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -113,6 +114,34 @@ typedef enum fa_dtype {
 fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
                  int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D,
                  fa_layout layout, int causal, float scale, fa_dtype dtype, void *stream);
+
+/*
+ * fa_fwd_ws -- fa_fwd with a dynamic work schedule: the same operation,
+ * arguments and results (bit-identical: each work unit is computed the same
+ * way), but the persistent CTAs take work units (two 128-row query tiles of
+ * one batch and head) from a counter in `workspace`, longest first, instead
+ * of a fixed round-robin share.  This balances causal workloads, whose units
+ * differ in length (page "64K long-sequence FlashAttention"
+ * (ai6s.net/6a140d07), section "multi-AI-Core load balancing": dynamic
+ * scheduling of uneven per-core tile counts).
+ *
+ * workspace        device memory of at least fa_fwd_workspace_size() bytes,
+ *                  16-byte aligned, owned by the caller; the library zeroes
+ *                  it on `stream` before the launch and uses it as scratch.
+ *                  It must not overlap any tensor argument, and two calls
+ *                  that may run at the same time need separate workspaces.
+ * workspace_bytes  its size in bytes.
+ *
+ * Errors as for fa_fwd, plus FA_ERR_INVALID_ARG (null or too small
+ * workspace), FA_ERR_MISALIGNED and FA_ERR_ALIAS for the workspace.
+ */
+fa_status fa_fwd_ws(const void *q, const void *k, const void *v, void *o, float *lse,
+                    int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D,
+                    fa_layout layout, int causal, float scale, fa_dtype dtype,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of device workspace fa_fwd_ws needs (a small constant). */
+size_t fa_fwd_workspace_size(void);
 
 /*
  * fa_device_status -- synchronises `stream`, then reads and clears the

@@ -131,3 +131,34 @@ def test_python_wrapper_checks_shapes():
     with pytest.raises(ValueError, match="contiguous"):
         t = torch.zeros(1, 2, 16, 64, dtype=torch.float16).transpose(1, 2)
         fa.flash_attention_forward(t, t, t, layout="BSND")
+
+
+WS = 0x60000000
+
+
+def call_ws(ws=WS, ws_bytes=16, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_fwd_ws(a.get("q", Q), a.get("k", K), a.get("v", V), a.get("o", O), a.get("lse", L),
+                        a["B"], a["H"], a["Sq"], a["Sk"], a["D"], a["layout"], a["causal"], a["scale"],
+                        a["dtype"], ws, ws_bytes, None)
+
+
+def test_workspace_size_is_small_constant(lib):
+    assert 4 <= fa.fa_fwd_workspace_size() <= 256
+    assert fa.fa_fwd_workspace_size() % 4 == 0
+
+
+def test_workspace_validation(lib):
+    assert call_ws(ws=0) == fa.FA_ERR_INVALID_ARG
+    assert call_ws(ws_bytes=fa.fa_fwd_workspace_size() - 1) == fa.FA_ERR_INVALID_ARG
+    assert call_ws(ws=WS + 4) == fa.FA_ERR_MISALIGNED
+    assert call_ws(ws=Q + 64) == fa.FA_ERR_ALIAS
+    assert call_ws(ws=L) == fa.FA_ERR_ALIAS
+    assert call_ws(ws=0, Sq=0) == fa.FA_OK
+    assert call_ws(D=96) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_dynamic_schedule_argument_errors_match_static(lib):
+    for kw in (dict(B=0), dict(layout=3), dict(dtype=5), dict(scale=float("nan"))):
+        assert call_ws(**kw) == call(**kw) == fa.FA_ERR_INVALID_ARG

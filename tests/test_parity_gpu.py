@@ -218,3 +218,36 @@ def test_stream_is_respected():
     torch.cuda.current_stream().wait_stream(s)
     fa.check_device_status(s)
     assert torch.equal(o, ref)
+
+
+SCHEDULE_CASES = [
+    W("bf16", "BHSD", 2, 40, 8192, 8192, 128, True),
+    W("bf16", "BSND", 1, 3, 1000, 1000, 128, True),
+    W("fp16", "BHSD", 2, 5, 700, 1900, 64, False),
+    W("bf16", "BHSD", 1, 8, 65536, 65536, 128, True),
+]
+
+
+@pytest.mark.parametrize("w", SCHEDULE_CASES, ids=lambda w: w.name)
+def test_static_and_dynamic_schedules_agree_bitwise(w):
+    """fa_fwd (static round-robin) and fa_fwd_ws (work counter) compute every
+    unit the same way, so their outputs are bit-identical."""
+    _need_gpu()
+    q, k, v = make_qkv(w, device="cuda")
+    o1, l1 = fa.flash_attention_forward(q, k, v, layout=w.layout, causal=w.causal, scale=w.scale, schedule="static")
+    o2, l2 = fa.flash_attention_forward(q, k, v, layout=w.layout, causal=w.causal, scale=w.scale, schedule="dynamic")
+    ws = torch.full((fa.fa_fwd_workspace_size(),), 255, dtype=torch.uint8, device="cuda")   # stale contents
+    o3, l3 = fa.flash_attention_forward(q, k, v, layout=w.layout, causal=w.causal, scale=w.scale, workspace=ws)
+    o4, l4 = fa.flash_attention_forward(q, k, v, layout=w.layout, causal=w.causal, scale=w.scale, workspace=ws)
+    fa.check_device_status()
+    for o, l in ((o2, l2), (o3, l3), (o4, l4)):
+        assert torch.equal(o1, o) and torch.equal(l1, l)
+
+
+def test_workspace_on_host_rejected():
+    _need_gpu()
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16, device="cuda")
+    host_ws = torch.zeros(fa.fa_fwd_workspace_size(), dtype=torch.uint8)
+    with pytest.raises(fa.FaError) as e:
+        fa.flash_attention_forward(q, q, q, layout="BHSD", workspace=host_ws)
+    assert e.value.status == fa.FA_ERR_NOT_DEVICE_POINTER
