@@ -36,8 +36,8 @@ FA_BF16 = 1
 LAYOUTS = {"BSND": FA_BSND, "BHSD": FA_BHSD}
 
 # Names every public symbol of include/fa_fwd.h.
-EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_device_status", "fa_query_support",
-                    "fa_status_string", "fa_last_cuda_error", "fa_version")
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_noalloc", "fa_device_status",
+                    "fa_query_support", "fa_status_string", "fa_last_cuda_error", "fa_version")
 
 
 class FaError(RuntimeError):
@@ -77,6 +77,8 @@ def load_library(path=None, rebuild_if_stale=True):
     lib.fa_fwd_ws.restype = c_int
     lib.fa_fwd_ws.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, vp,
                               ctypes.c_size_t, vp]
+    lib.fa_fwd_noalloc.restype = c_int
+    lib.fa_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, vp]
     lib.fa_fwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_fwd_workspace_size.argtypes = []
     lib.fa_device_status.restype = c_int
@@ -109,6 +111,14 @@ def fa_fwd_ws(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, wo
     lib = load_library()
     return lib.fa_fwd_ws(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
                          int(bool(causal)), float(scale), int(dtype), workspace, int(workspace_bytes), stream)
+
+
+def fa_fwd_noalloc(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, stream):
+    """The C fa_fwd_noalloc: the dynamic schedule with the library's fixed scratch, for callers
+    that cannot allocate device memory; returns the fa_status code."""
+    lib = load_library()
+    return lib.fa_fwd_noalloc(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
+                              int(bool(causal)), float(scale), int(dtype), stream)
 
 
 def fa_fwd_workspace_size():

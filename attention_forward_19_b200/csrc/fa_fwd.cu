@@ -1188,9 +1188,79 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
                           : launch<64, false>(prm, mq, mk, mv, mo, grid, &cfg[3], s);
 }
 
+// ---------------------------------------------------------------------------
+// Entry point without allocation (fa_fwd_noalloc).
+//
+// Some callers cannot give this library device memory: a plugin whose host
+// framework owns every device allocation and hands over only the input and
+// output buffers, or a real-time path that must not call the CUDA allocator
+// (cudaMalloc can synchronise the device and fragment a fixed memory budget).
+// For them the dynamic schedule's scratch -- its work counter -- lives in the
+// fixed array below, which every GPU that loads this library holds until the
+// process exits.  In host code the array's name is only a host-side stand-in;
+// its device address comes from cudaGetSymbolAddress, once per device, with
+// that device current, on the first fa_fwd_noalloc call there.
+constexpr size_t kNoAllocScratchBytes = 256;   // capacity of the fixed scratch
+static_assert(kWorkspaceBytes <= kNoAllocScratchBytes, "the fixed scratch cannot hold the schedule's counter");
+
+struct NoAllocScratch {
+  std::once_flag once;
+  void* ptr = nullptr;
+  int err = 0;
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char fa_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+// Device address of fa_noalloc_scratch on `dev` (the current device), looked
+// up on the first call for that device; nullptr with *err set on failure.
+void* noalloc_scratch_address(int dev, int* err) {
+  NoAllocScratch& slot = g_noalloc[dev];
+  std::call_once(slot.once, [&slot] {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, fa_noalloc_scratch);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      slot.err = (int)e;
+      return;
+    }
+    slot.ptr = ptr;
+  });
+  *err = slot.err;
+  return slot.ptr;
+}
+
 }  // namespace
 
 extern "C" {
+
+fa_status fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                         int64_t H, int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale,
+                         fa_dtype dtype, void* stream) {
+  // arguments that need no device, answered exactly as fa_fwd answers them
+  if (B <= 0 || H <= 0 || Sq < 0 || Sk <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
+  if (layout != FA_BSND && layout != FA_BHSD) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (Sq == 0) return FA_OK;
+  // the schedule needs kWorkspaceBytes of scratch whatever the sizes; a need
+  // beyond the fixed array is refused rather than overrun
+  if (kWorkspaceBytes > kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail((int)e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  int err = 0;
+  void* scratch = noalloc_scratch_address(dev, &err);
+  if (!scratch) return cuda_fail(err);
+  return fwd_impl(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype,
+                  static_cast<unsigned int*>(scratch), stream);
+}
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
                  int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,

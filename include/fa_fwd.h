@@ -144,6 +144,31 @@ fa_status fa_fwd_ws(const void *q, const void *k, const void *v, void *o, float 
 size_t fa_fwd_workspace_size(void);
 
 /*
+ * fa_fwd_noalloc -- fa_fwd_ws for callers that cannot allocate device memory.
+ * This entry point has no counterpart on the pages: it exists for callers
+ * that own only their input and output buffers -- a plugin inside a host
+ * framework that keeps every device allocation to itself, or a latency-bound
+ * path that must not call the CUDA allocator (cudaMalloc can synchronise the
+ * device and fragment a fixed memory budget).  It computes exactly what
+ * fa_fwd_ws computes and allocates nothing.
+ *
+ * The dynamic schedule's scratch (its work counter, 16 bytes) lives in a
+ * fixed 256-byte array inside the library, held by every GPU that loads the
+ * library until the process exits.  The first call on a device looks up that
+ * array's device address (cudaGetSymbolAddress, with the device current);
+ * make that first call before any stream capture.  Every call zeroes the
+ * counter on `stream` before its launch and then uses it, so calls that
+ * overlap on the same GPU (for example on two streams) race on it: serialise
+ * them, or use fa_fwd_ws with separate workspaces.  Each GPU has its own copy
+ * of the array.  Arguments, results and errors as for fa_fwd;
+ * FA_ERR_UNSUPPORTED if the schedule ever needed more scratch than the array
+ * holds.
+ */
+fa_status fa_fwd_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                         int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D,
+                         fa_layout layout, int causal, float scale, fa_dtype dtype, void *stream);
+
+/*
  * fa_device_status -- synchronises `stream`, then reads and clears the
  * library's device-side error word on the current device.  Returns FA_OK,
  * FA_ERR_TIMEOUT if a kernel stopped at a wait limit since the last call, or
