@@ -80,9 +80,15 @@ constexpr float RESCALE_LOG2 = FA_RESCALE_LOG2;  // O / l are rescaled only when
 constexpr float RESCALE_POW2 = (float)(1u << (int)FA_RESCALE_LOG2);  // 2^RESCALE_LOG2
 constexpr float HEADROOM_LOG2 = 8.0f;  // bf16 only: a moved reference sits this far above the tile max
 #ifndef FA_EMU_PAIRS
-#define FA_EMU_PAIRS 1
+#define FA_EMU_PAIRS 0
 #endif
-constexpr int EMU_PAIRS = FA_EMU_PAIRS;  // of every 4 exp2 pairs, this many run on the FMA pipe
+// Of the 64 exp2 pairs of a 128-key row, this many (spread evenly) run on the
+// FMA pipe.  The softmax loop is bound by instruction dispatch as much as by
+// MUFU: a MUFU pair costs 1 dispatch slot per value but 8 pipe cycles, an
+// emulated pair about 22 dispatch slots.  Measured on the workloads, 0 to 6
+// of 64 are within noise of each other and more is slower, so the default is 0.
+constexpr int EMU_PAIRS = FA_EMU_PAIRS;
+__host__ __device__ constexpr bool emulated_pair(int i, int e) { return (i * e) / 64 != ((i + 1) * e) / 64; }
 
 template <int D>
 struct Cfg {
@@ -430,6 +436,12 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
+__device__ __forceinline__ uint32_t imad_shl23(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // 2^x for two values on the FMA pipe instead of MUFU.  x = j + r with
 // j = round(x): adding 1.5 * 2^23 leaves j in the low mantissa bits, so
 // 1.5 * 2^23 - (x + 1.5 * 2^23) = -j exactly and r = x - j lies in [-1/2, 1/2].
@@ -462,8 +474,10 @@ __device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& y0, float& y1
   float p0, p1, t0, t1;
   f2unpack(p, p0, p1);
   f2unpack(t, t0, t1);
-  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+  // 2^j into the exponent field: bits(t) * 2^23 + bits(p) (an integer multiply-add,
+  // which runs on the FMA pipe); bits(t) * 2^23 keeps only j * 2^23 modulo 2^32
+  y0 = __uint_as_float(imad_shl23(__float_as_uint(t0), __float_as_uint(p0)));
+  y1 = __uint_as_float(imad_shl23(__float_as_uint(t1), __float_as_uint(p1)));
 }
 
 // max over the row of s * c (c > 0: max(s) * c; c < 0: min(s) * c; c = 0: 0).
@@ -489,8 +503,8 @@ __device__ __forceinline__ float row_max_scaled(const uint32_t (&sr)[BN], float 
   return fminf(fminf(a[0], a[1]), fminf(a[2], a[3])) * c;
 }
 
-// P = 2^(s * cc + neg_m) for the row: EMU of every 4 pairs on the FMA pipe,
-// the rest on MUFU; packed to the input dtype into pk (two per 32-bit word).
+// P = 2^(s * cc + neg_m) for the row: EMU of the 64 pairs (spread evenly) on
+// the FMA pipe, the rest on MUFU; packed to the input dtype into pk (two per 32-bit word).
 // Returns the fp32 row sum; ymax gets the largest fp32 weight (the one the
 // rounding correction is taken from, and the speculation check).
 template <bool BF16, int EMU>
@@ -503,7 +517,7 @@ __device__ __forceinline__ float exp_pack_row(const uint32_t (&sr)[BN], float cc
   for (int i = 0; i < BN / 2; ++i) {
     const uint64_t x2 = ffma2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), cc2, nm2);
     float y0, y1;
-    if ((i & 3) < EMU) {
+    if (emulated_pair(i, EMU)) {
       exp2_poly_pair<BF16 ? 3 : 4>(x2, y0, y1);
     } else {
       float x0, x1;
