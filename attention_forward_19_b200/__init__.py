@@ -36,8 +36,8 @@ FA_BF16 = 1
 LAYOUTS = {"BSND": FA_BSND, "BHSD": FA_BHSD}
 
 # Names every public symbol of include/fa_fwd.h.
-EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_noalloc", "fa_device_status",
-                    "fa_query_support", "fa_status_string", "fa_last_cuda_error", "fa_version")
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_noalloc", "fa_selftest_wait_timeout",
+                    "fa_device_status", "fa_query_support", "fa_status_string", "fa_last_cuda_error", "fa_version")
 
 
 class FaError(RuntimeError):
@@ -79,6 +79,9 @@ def load_library(path=None, rebuild_if_stale=True):
                               ctypes.c_size_t, vp]
     lib.fa_fwd_noalloc.restype = c_int
     lib.fa_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, vp]
+    lib.fa_selftest_wait_timeout.restype = c_int
+    lib.fa_selftest_wait_timeout.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float,
+                                             c_int, ctypes.c_uint32, vp]
     lib.fa_fwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_fwd_workspace_size.argtypes = []
     lib.fa_device_status.restype = c_int
@@ -119,6 +122,15 @@ def fa_fwd_noalloc(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtyp
     lib = load_library()
     return lib.fa_fwd_noalloc(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
                               int(bool(causal)), float(scale), int(dtype), stream)
+
+
+def fa_selftest_wait_timeout(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, wait_limit_us,
+                             stream):
+    """The C fa_selftest_wait_timeout: a launch whose loads are withheld, so that every bounded
+    wait runs out; returns the fa_status code of the launch."""
+    lib = load_library()
+    return lib.fa_selftest_wait_timeout(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
+                                        int(bool(causal)), float(scale), int(dtype), int(wait_limit_us), stream)
 
 
 def fa_fwd_workspace_size():

@@ -129,6 +129,7 @@ struct Params {
   int bhsd;            // 1: [B,H,S,D], 0: [B,S,H,D]
   float scale_log2;    // scale * log2(e)
   unsigned long long wait_limit_ns;
+  int withhold_loads;  // self-test of the bounded waits: the producer issues no loads
 };
 
 __device__ int g_dev_error = 0;
@@ -670,6 +671,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive(bar(C::UQ_FULL + qs));
         ++uq_pos;
         if (u >= p.total_units) break;
+        if (p.withhold_loads) {
+          // Self-test: nothing is loaded, so every consumer's wait for Q or
+          // K / V runs out, and nothing is in flight when the CTA drains.
+          u += (int)gridDim.x;
+          continue;
+        }
         const Unit un = decode_unit(p, u);
         const int n = max(un.n[0], un.n[1]);
 #pragma unroll
@@ -1111,9 +1118,14 @@ constexpr size_t kWorkspaceBytes = 16;  // the work counter of the dynamic sched
 // Validates the arguments, builds the tensor maps and launches the kernel.
 // sched: the dynamic-schedule counter in device memory (zeroed here, on the
 // stream, before the launch), or nullptr for the static schedule.
+// Self-test settings: a kernel that withholds its loads, with a short wait limit.
+struct SelfTest {
+  unsigned long long wait_limit_ns;
+};
+
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
                    int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
-                   unsigned int* sched, void* stream) {
+                   unsigned int* sched, void* stream, const SelfTest* selftest = nullptr) {
   // ---- arguments that need no device
   if (B <= 0 || H <= 0 || Sq < 0 || Sk <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
   if (layout != FA_BSND && layout != FA_BHSD) return FA_ERR_INVALID_ARG;
@@ -1186,6 +1198,11 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   prm.bhsd = layout == FA_BHSD ? 1 : 0;
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   prm.wait_limit_ns = 1000000000ull;  // one second; a normal wait lasts microseconds
+  prm.withhold_loads = 0;
+  if (selftest) {
+    prm.wait_limit_ns = selftest->wait_limit_ns;
+    prm.withhold_loads = 1;
+  }
 
   const int grid = (int)(prm.total_units < sms ? prm.total_units : sms);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -1305,6 +1322,14 @@ fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float*
 }
 
 size_t fa_fwd_workspace_size(void) { return kWorkspaceBytes; }
+
+fa_status fa_selftest_wait_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                                   int64_t H, int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal,
+                                   float scale, fa_dtype dtype, uint32_t wait_limit_us, void* stream) {
+  if (wait_limit_us < 1000u || wait_limit_us > 1000000u) return FA_ERR_INVALID_ARG;
+  const SelfTest st{(unsigned long long)wait_limit_us * 1000ull};
+  return fwd_impl(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, nullptr, stream, &st);
+}
 
 fa_status fa_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

@@ -144,6 +144,24 @@ fa_status fa_fwd_ws(const void *q, const void *k, const void *v, void *o, float 
 size_t fa_fwd_workspace_size(void);
 
 /*
+ * fa_selftest_wait_timeout -- exercises the kernel's failure detection
+ * without a fault.  The kernel is launched as by fa_fwd (same arguments and
+ * validation), but its producer warp issues no loads and every wait is limited
+ * to `wait_limit_us` microseconds (1,000 .. 1,000,000).  Every consumer's wait
+ * for Q or K / V therefore runs out; the CTAs record the timeout in the device
+ * error word, drain (nothing is in flight) and return.  q, k and v are not
+ * read; o and lse are not written.  Returns FA_OK once launched (or the
+ * argument error fa_fwd would return, FA_ERR_INVALID_ARG for a limit outside
+ * the range); the next fa_device_status() then returns FA_ERR_TIMEOUT and
+ * clears the word, and the CUDA context stays usable.  The pages have no
+ * counterpart: this is a test hook for the bounded waits.
+ */
+fa_status fa_selftest_wait_timeout(const void *q, const void *k, const void *v, void *o, float *lse,
+                                   int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D,
+                                   fa_layout layout, int causal, float scale, fa_dtype dtype,
+                                   uint32_t wait_limit_us, void *stream);
+
+/*
  * fa_fwd_noalloc -- fa_fwd_ws for callers that cannot allocate device memory.
  * This entry point has no counterpart on the pages: it exists for callers
  * that own only their input and output buffers -- a plugin inside a host

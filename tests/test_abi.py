@@ -162,3 +162,20 @@ def test_workspace_validation(lib):
 def test_dynamic_schedule_argument_errors_match_static(lib):
     for kw in (dict(B=0), dict(layout=3), dict(dtype=5), dict(scale=float("nan"))):
         assert call_ws(**kw) == call(**kw) == fa.FA_ERR_INVALID_ARG
+
+
+def call_selftest(limit_us=20000, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_selftest_wait_timeout(Q, K, V, O, L, a["B"], a["H"], a["Sq"], a["Sk"], a["D"], a["layout"],
+                                       a["causal"], a["scale"], a["dtype"], limit_us, None)
+
+
+def test_selftest_limit_range_and_argument_checks(lib):
+    """The wait-timeout self-test takes a limit of 1 ms .. 1 s and validates like fa_fwd."""
+    assert call_selftest(limit_us=999) == fa.FA_ERR_INVALID_ARG
+    assert call_selftest(limit_us=1000001) == fa.FA_ERR_INVALID_ARG
+    for kw in (dict(B=0), dict(layout=3), dict(dtype=5), dict(scale=float("nan"))):
+        assert call_selftest(**kw) == call(**kw) == fa.FA_ERR_INVALID_ARG
+    assert call_selftest(D=96) == fa.FA_ERR_UNSUPPORTED
+    assert call_selftest(Sq=0) == fa.FA_OK

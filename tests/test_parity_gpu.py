@@ -45,6 +45,7 @@ def compare_full(orc, w, q, k, v, o, lse, scale=None):
     lse_gpu = lse.cpu().to(torch.float64).numpy()
     eo = np.max(np.abs(o_gpu - o_ref))
     el = np.max(np.abs(lse_gpu - lse_ref))
+    print(f"PARITY {w.name}: max|dO| {eo:.3e} max|dLSE| {el:.3e} ({o_gpu.shape[0] if o_gpu.ndim == 2 else 'all'} rows)")
     assert np.all(np.isfinite(o_gpu)) and np.all(np.isfinite(lse_gpu))
     assert eo <= O_TOL[w.dtype], f"{w.name}: max |dO| = {eo}"
     assert el <= LSE_TOL, f"{w.name}: max |dLSE| = {el}"
@@ -61,6 +62,7 @@ def compare_rows(orc, w, q, k, v, o, lse, rows):
     lse_gpu = lse.reshape(-1).index_select(0, idx).cpu().to(torch.float64).numpy()
     eo = np.max(np.abs(o_gpu - o_ref))
     el = np.max(np.abs(lse_gpu - lse_ref))
+    print(f"PARITY {w.name}: max|dO| {eo:.3e} max|dLSE| {el:.3e} ({o_gpu.shape[0] if o_gpu.ndim == 2 else 'all'} rows)")
     assert np.all(np.isfinite(o_gpu)) and np.all(np.isfinite(lse_gpu))
     assert eo <= O_TOL[w.dtype], f"{w.name}: max |dO| = {eo} over {len(rows)} rows"
     assert el <= LSE_TOL, f"{w.name}: max |dLSE| = {el} over {len(rows)} rows"
