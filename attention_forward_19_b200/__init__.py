@@ -36,8 +36,9 @@ FA_BF16 = 1
 LAYOUTS = {"BSND": FA_BSND, "BHSD": FA_BHSD}
 
 # Names every public symbol of include/fa_fwd.h.
-EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_noalloc", "fa_selftest_wait_timeout",
-                    "fa_device_status", "fa_query_support", "fa_status_string", "fa_last_cuda_error", "fa_version")
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_noalloc", "fa_fwd_varlen",
+                    "fa_selftest_wait_timeout", "fa_device_status", "fa_query_support", "fa_status_string",
+                    "fa_last_cuda_error", "fa_version")
 
 
 class FaError(RuntimeError):
@@ -79,6 +80,9 @@ def load_library(path=None, rebuild_if_stale=True):
                               ctypes.c_size_t, vp]
     lib.fa_fwd_noalloc.restype = c_int
     lib.fa_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, vp]
+    lib.fa_fwd_varlen.restype = c_int
+    lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, c_int, c_float,
+                                  c_int, vp, ctypes.c_size_t, vp]
     lib.fa_selftest_wait_timeout.restype = c_int
     lib.fa_selftest_wait_timeout.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float,
                                              c_int, ctypes.c_uint32, vp]
@@ -122,6 +126,15 @@ def fa_fwd_noalloc(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtyp
     lib = load_library()
     return lib.fa_fwd_noalloc(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
                               int(bool(causal)), float(scale), int(dtype), stream)
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, H, total_q, total_k, max_q, max_k, D, causal, scale, dtype,
+                  workspace, workspace_bytes, stream):
+    """The C fa_fwd_varlen (packed variable-length batch) with raw pointers; returns the fa_status code."""
+    lib = load_library()
+    return lib.fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, int(B), int(H), int(total_q), int(total_k), int(max_q),
+                             int(max_k), int(D), int(bool(causal)), float(scale), int(dtype), workspace,
+                             int(workspace_bytes), stream)
 
 
 def fa_selftest_wait_timeout(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, wait_limit_us,
@@ -243,8 +256,76 @@ def flash_attention_forward(q, k, v, layout="BSND", causal=False, scale=None, he
     return out, lse
 
 
+def flash_attention_varlen_forward(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q=None, max_seqlen_k=None,
+                                   causal=False, scale=None, out=None, lse=None, stream=None, schedule="dynamic",
+                                   workspace=None):
+    """Attention forward over a packed batch of sequences of different lengths.
+
+    q: [total_q, H, D]; k, v: [total_k, H, D]; cu_seqlens_q / cu_seqlens_k: int32
+    CUDA tensors of B + 1 offsets (sequence b owns rows cu[b] .. cu[b+1]-1).
+    max_seqlen_q / max_seqlen_k bound the lengths; when None they are read from
+    the offsets (a device-to-host copy, which synchronises).  Returns (o, lse):
+    o like q, lse fp32 [H, total_q].  Invalid offsets are reported by
+    check_device_status().
+    """
+    import torch
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape:
+        raise ValueError("q must be [total_q, H, D] and k, v [total_k, H, D]")
+    total_q, H, D = q.shape
+    total_k, Hk, Dk = k.shape
+    if (Hk, Dk) != (H, D):
+        raise ValueError(f"q {tuple(q.shape)} and k {tuple(k.shape)} differ in heads or head dim")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.dtype != q.dtype:
+            raise TypeError("q, k, v must share one dtype")
+    for name, c in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if c.dtype != torch.int32 or c.dim() != 1 or not c.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 1-D int32 tensor")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must hold the same number (B + 1 >= 2) of offsets")
+    B = cu_seqlens_q.numel() - 1
+    if max_seqlen_q is None:
+        max_seqlen_q = int((cu_seqlens_q[1:] - cu_seqlens_q[:-1]).max().item())
+    if max_seqlen_k is None:
+        max_seqlen_k = int((cu_seqlens_k[1:] - cu_seqlens_k[:-1]).max().item())
+    dt = _dtype_code(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    if out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor like q")
+    if lse.shape != (H, total_q) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 tensor of shape [H, total_q]")
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device) if q.is_cuda else None
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    ws_ptr, ws_bytes = None, 0
+    if schedule == "dynamic":
+        nbytes = fa_fwd_workspace_size()
+        if workspace is None:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+        ws_bytes = workspace.numel() * workspace.element_size()
+        if ws_bytes < nbytes or not workspace.is_contiguous():
+            raise ValueError(f"workspace must be a contiguous tensor of at least {nbytes} bytes")
+        ws_ptr = workspace.data_ptr()
+    elif schedule != "static":
+        raise ValueError(f"schedule must be 'dynamic' or 'static', not {schedule!r}")
+    st = fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                       cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, H, total_q, total_k, max_seqlen_q,
+                       max_seqlen_k, D, causal, scale, dt, ws_ptr, ws_bytes, sptr)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_varlen")
+    return out, lse
+
+
 def check_device_status(stream=None):
-    """Synchronises the stream and raises FaError if a kernel reported a wait timeout."""
+    """Synchronises the stream and raises FaError if a kernel reported a wait timeout (or invalid
+    sequence offsets of a variable-length batch)."""
     import torch
     if stream is None:
         stream = torch.cuda.current_stream()

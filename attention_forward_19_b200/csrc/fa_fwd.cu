@@ -119,7 +119,7 @@ struct Cfg {
 struct Params {
   float* lse;
   unsigned int* sched;  // work counter for the dynamic schedule (zeroed before launch), or nullptr: static
-  int B, H, Sq, Sk;
+  int B, H, Sq, Sk;      // variable-length batch: Sq, Sk = the longest sequence
   int nqb;             // query units per head: ceil(Sq / 256)
   int tk;              // key tiles: ceil(Sk / 128)
   int bh;              // B * H
@@ -130,8 +130,17 @@ struct Params {
   float scale_log2;    // scale * log2(e)
   unsigned long long wait_limit_ns;
   int withhold_loads;  // self-test of the bounded waits: the producer issues no loads
+  // Variable-length batch (packed [total, H, D] rows), else cu_q == nullptr:
+  // sequence b has query rows [cu_q[b], cu_q[b+1]) and keys [cu_k[b], cu_k[b+1]).
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
+  uint8_t* o;           // O base (variable-length batch: rows of a ragged last tile are stored directly)
+  long long lse_bs, lse_hs;   // LSE offsets of a batch and of a head (plus the packed row)
 };
 
+// Device error word: bit 0 a wait ran out (FA_ERR_TIMEOUT), bit 1 invalid
+// sequence offsets of a variable-length batch (FA_ERR_INVALID_ARG).
 __device__ int g_dev_error = 0;
 
 // ----------------------------------------------------------------------------- PTX helpers
@@ -187,7 +196,7 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
       if (*abort_flag) break;
       if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
-        atomicExch(&g_dev_error, 1);
+        atomicOr(&g_dev_error, 1);
         break;
       }
     }
@@ -207,7 +216,7 @@ __device__ __forceinline__ bool wait_bar1(uint32_t bar, uint32_t parity, volatil
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
-      atomicExch(&g_dev_error, 1);
+      atomicOr(&g_dev_error, 1);
       return false;
     }
   }
@@ -219,7 +228,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > limit_ns) {
-      atomicExch(&g_dev_error, 1);
+      atomicOr(&g_dev_error, 1);
       return;
     }
   }
@@ -555,13 +564,17 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, uint32_t fmt, uin
 // ----------------------------------------------------------------------------- schedule
 
 struct Unit {
-  int b, h, r0;     // batch, head, first query row of the unit
+  int b, h, r0;     // batch, head, first query row of the unit (within its sequence)
   int rows[NQ];     // valid rows of each query tile
   int n[NQ];        // key tiles each query tile visits (0: tile inactive)
+  int sq, sk;       // the sequence's query and key lengths
+  int rb, kb;       // its first packed query row and key row (0 for a dense batch)
+  int tb;           // batch coordinate of the tensor maps (0 for a packed batch)
 };
 
 // Units are grouped by heads so that the K / V of a group stay in L2; inside
 // a group the longest units (causal: the last query rows) come first.
+template <bool VARLEN>
 __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
   const int per_group = p.group_heads * p.nqb;
   const int g = u / per_group;
@@ -574,18 +587,38 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
   un.b = bh / p.H;
   un.h = bh - un.b * p.H;
   un.r0 = qblk * UNIT_ROWS;
+  if constexpr (VARLEN) {
+    // Every role decodes the same offsets.  Offsets that cannot describe a
+    // sequence of this batch (and a sequence with queries but no keys) make
+    // the unit empty and are reported in the device error word.
+    const int q0 = p.cu_q[un.b], q1 = p.cu_q[un.b + 1], k0 = p.cu_k[un.b], k1 = p.cu_k[un.b + 1];
+    const bool bad = q0 < 0 || q1 < q0 || q1 > p.total_q || q1 - q0 > p.Sq || k0 < 0 || k1 < k0 ||
+                     k1 > p.total_k || k1 - k0 > p.Sk || (k1 == k0 && q1 > q0);
+    if (bad && un.r0 == 0) atomicOr(&g_dev_error, 2);
+    un.sq = bad ? 0 : q1 - q0;
+    un.sk = bad ? 0 : k1 - k0;
+    un.rb = q0;
+    un.kb = k0;
+    un.tb = 0;
+  } else {
+    un.sq = p.Sq;
+    un.sk = p.Sk;
+    un.rb = 0;
+    un.kb = 0;
+    un.tb = un.b;
+  }
 #pragma unroll
   for (int t = 0; t < NQ; ++t) {
     const int first = un.r0 + t * BM;
-    const int rows = max(0, min(BM, p.Sq - first));
+    const int rows = max(0, min(BM, un.sq - first));
     un.rows[t] = rows;
     if (rows == 0) {
       un.n[t] = 0;
     } else if (p.causal) {
-      const int last_key = min(first + rows - 1, p.Sk - 1);
+      const int last_key = min(first + rows - 1, un.sk - 1);
       un.n[t] = last_key / BN + 1;
     } else {
-      un.n[t] = p.tk;
+      un.n[t] = (un.sk + BN - 1) / BN;
     }
   }
   return un;
@@ -593,7 +626,7 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
 
 // ----------------------------------------------------------------------------- kernel
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool VARLEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -677,7 +710,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           u += (int)gridDim.x;
           continue;
         }
-        const Unit un = decode_unit(p, u);
+        const Unit un = decode_unit<VARLEN>(p, u);
         const int n = max(un.n[0], un.n[1]);
 #pragma unroll
         for (int t = 0; t < NQ; ++t) {
@@ -686,10 +719,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!ok) break;
           ++q_use[t];
           mbar_arrive_expect_tx(bar(C::Q_FULL + t), C::TILE_BYTES);
-          const int s0 = un.r0 + t * BM;
+          const int s0 = un.rb + un.r0 + t * BM;
           for (int bx = 0; bx < C::NBOX; ++bx)
             tma_load_4d(sQ + t * C::TILE_BYTES + bx * BOX_BYTES, &tmQ, bar(C::Q_FULL + t), bx * 64,
-                        p.bhsd ? s0 : un.h, p.bhsd ? un.h : s0, un.b);
+                        p.bhsd ? s0 : un.h, p.bhsd ? un.h : s0, un.tb);
         }
         for (int j = 0; j < n && ok; ++j) {
           for (int kv = 0; kv < 2; ++kv) {
@@ -699,10 +732,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!ok) break;
             mbar_arrive_expect_tx(bar(C::KV_FULL + slot), C::TILE_BYTES);
             const CUtensorMap* map = kv ? &tmV : &tmK;
-            const int s0 = j * BN;
+            const int s0 = un.kb + j * BN;
             for (int bx = 0; bx < C::NBOX; ++bx)
               tma_load_4d(sKV + slot * C::TILE_BYTES + bx * BOX_BYTES, map, bar(C::KV_FULL + slot),
-                          bx * 64, p.bhsd ? s0 : un.h, p.bhsd ? un.h : s0, un.b);
+                          bx * 64, p.bhsd ? s0 : un.h, p.bhsd ? un.h : s0, un.tb);
             ++kv_cnt;
           }
         }
@@ -760,8 +793,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) mbar_arrive(bar(C::UQ_EMPTY + qs));
       ++uq_pos;
       if (u >= p.total_units) break;
-      const Unit un = decode_unit(p, u);
+      const Unit un = decode_unit<VARLEN>(p, u);
       const int n = max(un.n[0], un.n[1]);
+      if (VARLEN && n == 0) continue;   // an empty sequence of a variable-length batch
 #pragma unroll
       for (int t = 0; t < NQ; ++t) {
         if (un.n[t] == 0 || !ok) continue;
@@ -780,6 +814,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (un.n[t] == 0) continue;
         qk(t, kslot);
         tc_commit_elect(bar(C::S_FULL + t));
+        // packed batch: Q_t is read by no later MMA, so the producer may load
+        // the next unit's Q_t as soon as this one completes
+        if (VARLEN && un.n[t] == 1) tc_commit_elect(bar(C::Q_EMPTY + t));
       }
       tc_commit_elect(bar(C::KV_EMPTY + kslot));
       for (int j = 0; j < n && ok; ++j) {
@@ -816,6 +853,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // softmax may rescale O_t once it has seen S_t(j+1).
             qk(t, kslot);
             tc_commit_elect(bar(C::S_FULL + t));
+            if (VARLEN && j + 2 == un.n[t]) tc_commit_elect(bar(C::Q_EMPTY + t));   // last read of Q_t
           }
         }
         if (!ok) break;
@@ -852,7 +890,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) mbar_arrive(bar(C::UQ_EMPTY + qs));
       ++uq_pos;
       if (u >= p.total_units) break;
-      const Unit un = decode_unit(p, u);
+      const Unit un = decode_unit<VARLEN>(p, u);
       const int nt = t ? un.n[1] : un.n[0];
       if (nt == 0) continue;
       const int row = un.r0 + t * BM + rit;          // query row of this thread
@@ -868,9 +906,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++s_use;
         tc_fence_after();
         const int c0 = j * BN;
-        const bool masked = (c0 + BN > p.Sk) || (p.causal && (c0 + BN - 1 > first_row));
+        const bool masked = (c0 + BN > un.sk) || (p.causal && (c0 + BN - 1 > first_row));
         const float cc = masked ? 1.f : c;
-        int lim = p.Sk - 1 - c0;
+        int lim = un.sk - 1 - c0;
         if (p.causal) lim = min(lim, row - c0);
         // this row of S_t from TMEM; diagonal / ragged tiles become scaled logits
         // with masked entries at -inf
@@ -953,6 +991,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ++o_use;
       tc_fence_after();
       const float inv_l = 1.f / ln;
+      // Dense batch: O is staged (swizzled) in the Q tile's buffer and stored
+      // by TMA; the buffer is released once the store has read it.  Packed
+      // (variable-length) batch: each thread stores its own row from
+      // registers -- a tile may end inside the sequence, where a TMA store
+      // would also write the next sequence's rows -- and the MMA warp has
+      // already released the Q buffer after its last read.
+      const bool store_row = row < un.sq;
+      uint8_t* orow = nullptr;
+      if constexpr (VARLEN) orow = p.o + ((size_t)(un.rb + row) * p.H + un.h) * (D * 2);
       {
         uint32_t r[32];
 #pragma unroll
@@ -964,38 +1011,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
-          // row rit of box q4/2, 16-byte chunks (q4&1)*4 + i, 128-byte swizzle
-          uint8_t* rowp = sQt + (q4 >> 1) * BOX_BYTES + rit * 128;
+          if constexpr (VARLEN) {
+            if (store_row) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 64);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int chunk = ((q4 & 1) * 4 + i) ^ (rit & 7);
-            *reinterpret_cast<uint4*>(rowp + chunk * 16) = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+          } else {
+            // row rit of box q4/2, 16-byte chunks (q4&1)*4 + i, 128-byte swizzle
+            uint8_t* rowp = sQt + (q4 >> 1) * BOX_BYTES + rit * 128;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int chunk = ((q4 & 1) * 4 + i) ^ (rit & 7);
+              *reinterpret_cast<uint4*>(rowp + chunk * 16) =
+                  make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
           }
         }
       }
       tc_fence_before();
       mbar_arrive(bar(C::O_EMPTY + t));
-      fence_proxy_async_smem();
-      mbar_arrive(bar(C::EPI + t));
-      if (row < p.Sq) {
+      if constexpr (!VARLEN) {
+        fence_proxy_async_smem();
+        mbar_arrive(bar(C::EPI + t));
+      }
+      if (store_row) {
         const float lse = (m_use + lg2(l)) * 0.69314718055994530942f;
-        p.lse[((size_t)(un.b * p.H + un.h)) * p.Sq + row] = lse;
+        p.lse[(size_t)un.b * p.lse_bs + (size_t)un.h * p.lse_hs + un.rb + row] = lse;
       }
-      if (rit == 0) {
-        // one thread stores the tile once all 128 rows are staged
-        drain_wait(bar(C::EPI + t), e_use & 1u, limit);
-        const int s0 = first_row;
-        for (int bx = 0; bx < C::NBOX; ++bx)
-          tma_store_4d(&tmO, smem_u32(sQt + bx * BOX_BYTES), bx * 64, p.bhsd ? s0 : un.h,
-                       p.bhsd ? un.h : s0, un.b);
-        tma_store_commit();
-        tma_store_wait_read();
-        mbar_arrive(bar(C::Q_EMPTY + t));
+      if constexpr (!VARLEN) {
+        if (rit == 0) {
+          // one thread stores the tile once all 128 rows are staged
+          drain_wait(bar(C::EPI + t), e_use & 1u, limit);
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_store_4d(&tmO, smem_u32(sQt + bx * BOX_BYTES), bx * 64, p.bhsd ? first_row : un.h,
+                         p.bhsd ? un.h : first_row, un.tb);
+          tma_store_commit();
+          tma_store_wait_read();
+          mbar_arrive(bar(C::Q_EMPTY + t));
+        }
+        ++e_use;
       }
-      ++e_use;
       __syncwarp();
     }
-    if (rit == 0) tma_store_wait_all();
+    if constexpr (!VARLEN) {
+      if (rit == 0) tma_store_wait_all();
+    }
     __syncwarp();
   }
 
@@ -1090,13 +1151,13 @@ fa_status check_device_ptr(const void* ptr, int device) {
 
 struct DeviceInfo {
   int sms = 0;
-  bool configured[4] = {false, false, false, false};
+  bool configured[8] = {false, false, false, false, false, false, false, false};
 };
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool VARLEN>
 fa_status launch(const fa::Params& prm, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                  const CUtensorMap& o, int grid, bool* configured, cudaStream_t stream) {
-  auto kern = fa::fa_fwd_kernel<D, BF16>;
+  auto kern = fa::fa_fwd_kernel<D, BF16, VARLEN>;
   const int smem = fa::Cfg<D>::SMEM_BYTES;
   if (!*configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1118,6 +1179,62 @@ constexpr size_t kWorkspaceBytes = 16;  // the work counter of the dynamic sched
 // Validates the arguments, builds the tensor maps and launches the kernel.
 // sched: the dynamic-schedule counter in device memory (zeroed here, on the
 // stream, before the launch), or nullptr for the static schedule.
+// The current device, its SM count, and every non-null pointer on it.
+fa_status device_checks(const void* const* ptrs, int n, int* dev_out, int* sms_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail((int)e);
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  for (int i = 0; i < n; ++i) {
+    if (!ptrs[i]) continue;   // optional arguments (the work counter) may be null
+    fa_status st = check_device_ptr(ptrs[i], dev);
+    if (st != FA_OK) return st;
+  }
+  std::lock_guard<std::mutex> g(g_dev_mu);
+  if (g_dev[dev].sms == 0) {
+    e = cudaDeviceGetAttribute(&g_dev[dev].sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail((int)e);
+  }
+  *dev_out = dev;
+  *sms_out = g_dev[dev].sms;
+  return FA_OK;
+}
+
+// Persistent grid of min(#SMs, #units) CTAs; zeroes the work counter first.
+fa_status launch_units(fa::Params& prm, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const CUtensorMap& mo, int64_t D, fa_dtype dtype, unsigned int* sched, int dev, int sms,
+                       void* stream) {
+  const int grid = (int)(prm.total_units < sms ? prm.total_units : sms);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  prm.sched = sched;
+  if (sched) {
+    cudaError_t e = cudaMemsetAsync(sched, 0, sizeof(unsigned int), s);
+    if (e != cudaSuccess) return cuda_fail((int)e);
+  }
+  bool* cfg = g_dev[dev].configured;
+  if (prm.cu_q) {
+    if (D == 128)
+      return dtype == FA_BF16 ? launch<128, true, true>(prm, mq, mk, mv, mo, grid, &cfg[4], s)
+                              : launch<128, false, true>(prm, mq, mk, mv, mo, grid, &cfg[5], s);
+    return dtype == FA_BF16 ? launch<64, true, true>(prm, mq, mk, mv, mo, grid, &cfg[6], s)
+                            : launch<64, false, true>(prm, mq, mk, mv, mo, grid, &cfg[7], s);
+  }
+  if (D == 128)
+    return dtype == FA_BF16 ? launch<128, true, false>(prm, mq, mk, mv, mo, grid, &cfg[0], s)
+                            : launch<128, false, false>(prm, mq, mk, mv, mo, grid, &cfg[1], s);
+  return dtype == FA_BF16 ? launch<64, true, false>(prm, mq, mk, mv, mo, grid, &cfg[2], s)
+                          : launch<64, false, false>(prm, mq, mk, mv, mo, grid, &cfg[3], s);
+}
+
+// Heads whose K and V (Sk keys each) fit together in about 48 MB of L2.
+int l2_group_heads(int64_t Sk, int64_t D, int64_t BH) {
+  const int64_t kv_head_bytes = 2 * Sk * D * 2;
+  int64_t gh = ((int64_t)48 << 20) / (kv_head_bytes > 0 ? kv_head_bytes : 1);
+  if (gh < 1) gh = 1;
+  if (gh > BH) gh = BH;
+  return (int)gh;
+}
+
 // Self-test settings: a kernel that withholds its loads, with a short wait limit.
 struct SelfTest {
   unsigned long long wait_limit_ns;
@@ -1151,28 +1268,12 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     return FA_ERR_ALIAS;
 
   // ---- device checks
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail((int)e);
-  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  int dev = 0, sms = 0;
   const void* ptrs[6] = {q, k, v, o, lse, sched};
-  for (const void* ptr : ptrs) {
-    if (!ptr) continue;   // only sched may be null here
-    fa_status st = check_device_ptr(ptr, dev);
-    if (st != FA_OK) return st;
-  }
-  int sms;
-  {
-    std::lock_guard<std::mutex> g(g_dev_mu);
-    if (g_dev[dev].sms == 0) {
-      e = cudaDeviceGetAttribute(&g_dev[dev].sms, cudaDevAttrMultiProcessorCount, dev);
-      if (e != cudaSuccess) return cuda_fail((int)e);
-    }
-    sms = g_dev[dev].sms;
-  }
+  fa_status st = device_checks(ptrs, 6, &dev, &sms);
+  if (st != FA_OK) return st;
 
   CUtensorMap mq, mk, mv, mo;
-  fa_status st;
   if ((st = make_map(&mq, q, dtype, layout, B, H, Sq, D)) != FA_OK) return st;
   if ((st = make_map(&mk, k, dtype, layout, B, H, Sk, D)) != FA_OK) return st;
   if ((st = make_map(&mv, v, dtype, layout, B, H, Sk, D)) != FA_OK) return st;
@@ -1180,6 +1281,13 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
 
   fa::Params prm;
   prm.lse = lse;
+  prm.cu_q = nullptr;
+  prm.cu_k = nullptr;
+  prm.total_q = 0;
+  prm.total_k = 0;
+  prm.o = static_cast<uint8_t*>(o);
+  prm.lse_bs = H * Sq;
+  prm.lse_hs = Sq;
   prm.B = (int)B;
   prm.H = (int)H;
   prm.Sq = (int)Sq;
@@ -1187,12 +1295,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   prm.nqb = (int)nqb;
   prm.tk = (int)((Sk + fa::BN - 1) / fa::BN);
   prm.bh = (int)(B * H);
-  // heads whose K and V fit together in about 48 MB of L2
-  const int64_t kv_head_bytes = 2 * Sk * D * 2;
-  int64_t gh = ((int64_t)48 << 20) / (kv_head_bytes > 0 ? kv_head_bytes : 1);
-  if (gh < 1) gh = 1;
-  if (gh > B * H) gh = B * H;
-  prm.group_heads = (int)gh;
+  prm.group_heads = l2_group_heads(Sk, D, B * H);
   prm.total_units = (int)(B * H * nqb);
   prm.causal = causal ? 1 : 0;
   prm.bhsd = layout == FA_BHSD ? 1 : 0;
@@ -1204,19 +1307,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
     prm.withhold_loads = 1;
   }
 
-  const int grid = (int)(prm.total_units < sms ? prm.total_units : sms);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  prm.sched = sched;
-  if (sched) {
-    e = cudaMemsetAsync(sched, 0, sizeof(unsigned int), s);
-    if (e != cudaSuccess) return cuda_fail((int)e);
-  }
-  bool* cfg = g_dev[dev].configured;
-  if (D == 128)
-    return dtype == FA_BF16 ? launch<128, true>(prm, mq, mk, mv, mo, grid, &cfg[0], s)
-                            : launch<128, false>(prm, mq, mk, mv, mo, grid, &cfg[1], s);
-  return dtype == FA_BF16 ? launch<64, true>(prm, mq, mk, mv, mo, grid, &cfg[2], s)
-                          : launch<64, false>(prm, mq, mk, mv, mo, grid, &cfg[3], s);
+  return launch_units(prm, mq, mk, mv, mo, D, dtype, sched, dev, sms, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -1323,6 +1414,87 @@ fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float*
 
 size_t fa_fwd_workspace_size(void) { return kWorkspaceBytes; }
 
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
+                        const int32_t* cu_seqlens_k, int64_t B, int64_t H, int64_t total_q, int64_t total_k,
+                        int64_t max_seqlen_q, int64_t max_seqlen_k, int64_t D, int causal, float scale,
+                        fa_dtype dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  // ---- arguments that need no device
+  if (B <= 0 || H <= 0 || D <= 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
+    return FA_ERR_INVALID_ARG;
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  const int64_t lim = (int64_t)1 << 30;
+  if (B >= lim || H >= lim || total_q >= lim || total_k >= lim || B * H >= lim) return FA_ERR_UNSUPPORTED;
+  if (max_seqlen_q > total_q || max_seqlen_k > total_k) return FA_ERR_INVALID_ARG;
+  const int64_t nqb = (max_seqlen_q + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+  if (B * H * nqb >= lim) return FA_ERR_UNSUPPORTED;
+  if (total_q == 0 || max_seqlen_q == 0) return FA_OK;   // no query rows
+  if (max_seqlen_k == 0) return FA_ERR_INVALID_ARG;      // queries without keys
+  if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
+       reinterpret_cast<uintptr_t>(o)) & 15u)
+    return FA_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(lse) | reinterpret_cast<uintptr_t>(cu_seqlens_q) |
+       reinterpret_cast<uintptr_t>(cu_seqlens_k)) & 3u)
+    return FA_ERR_MISALIGNED;
+  if (workspace) {
+    if (workspace_bytes < kWorkspaceBytes) return FA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return FA_ERR_MISALIGNED;
+  }
+  const size_t qbytes = (size_t)(total_q * H * D) * 2, kvbytes = (size_t)(total_k * H * D) * 2;
+  const size_t lbytes = (size_t)(total_q * H) * 4, cbytes = (size_t)(B + 1) * 4;
+  const void* outs[2] = {o, lse};
+  const size_t out_bytes[2] = {qbytes, lbytes};
+  const void* ins[6] = {q, k, v, cu_seqlens_q, cu_seqlens_k, workspace};
+  const size_t in_bytes[6] = {qbytes, kvbytes, kvbytes, cbytes, cbytes, workspace_bytes};
+  for (int i = 0; i < 2; ++i)
+    for (int j = 0; j < 6; ++j)
+      if (ins[j] && overlaps(outs[i], out_bytes[i], ins[j], in_bytes[j])) return FA_ERR_ALIAS;
+  if (overlaps(o, qbytes, lse, lbytes)) return FA_ERR_ALIAS;
+  if (workspace)
+    for (int j = 0; j < 5; ++j)
+      if (overlaps(workspace, workspace_bytes, ins[j], in_bytes[j])) return FA_ERR_ALIAS;
+
+  // ---- device checks
+  int dev = 0, sms = 0;
+  const void* ptrs[8] = {q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, workspace};
+  fa_status st = device_checks(ptrs, 8, &dev, &sms);
+  if (st != FA_OK) return st;
+
+  // packed rows [total, H, D] are the BSND layout with one batch entry
+  CUtensorMap mq, mk, mv, mo;
+  if ((st = make_map(&mq, q, dtype, FA_BSND, 1, H, total_q, D)) != FA_OK) return st;
+  if ((st = make_map(&mk, k, dtype, FA_BSND, 1, H, total_k, D)) != FA_OK) return st;
+  if ((st = make_map(&mv, v, dtype, FA_BSND, 1, H, total_k, D)) != FA_OK) return st;
+  if ((st = make_map(&mo, o, dtype, FA_BSND, 1, H, total_q, D)) != FA_OK) return st;
+
+  fa::Params prm;
+  prm.lse = lse;
+  prm.cu_q = cu_seqlens_q;
+  prm.cu_k = cu_seqlens_k;
+  prm.total_q = (int)total_q;
+  prm.total_k = (int)total_k;
+  prm.o = static_cast<uint8_t*>(o);
+  prm.lse_bs = 0;
+  prm.lse_hs = total_q;
+  prm.B = (int)B;
+  prm.H = (int)H;
+  prm.Sq = (int)max_seqlen_q;
+  prm.Sk = (int)max_seqlen_k;
+  prm.nqb = (int)nqb;
+  prm.tk = (int)((max_seqlen_k + fa::BN - 1) / fa::BN);
+  prm.bh = (int)(B * H);
+  prm.group_heads = l2_group_heads(max_seqlen_k, D, B * H);
+  prm.total_units = (int)(B * H * nqb);
+  prm.causal = causal ? 1 : 0;
+  prm.bhsd = 0;
+  prm.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  prm.wait_limit_ns = 1000000000ull;
+  prm.withhold_loads = 0;
+  return launch_units(prm, mq, mk, mv, mo, D, dtype, static_cast<unsigned int*>(workspace), dev, sms, stream);
+}
+
 fa_status fa_selftest_wait_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
                                    int64_t H, int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal,
                                    float scale, fa_dtype dtype, uint32_t wait_limit_us, void* stream) {
@@ -1341,7 +1513,7 @@ fa_status fa_device_status(void* stream) {
     const int zero = 0;
     e = cudaMemcpyToSymbol(fa::g_dev_error, &zero, sizeof(int));
     if (e != cudaSuccess) return cuda_fail((int)e);
-    return FA_ERR_TIMEOUT;
+    return (v & 1) ? FA_ERR_TIMEOUT : FA_ERR_INVALID_ARG;
   }
   return FA_OK;
 }

@@ -100,3 +100,72 @@ def sample_rows(w: Workload, per_head_first=64, per_head_last=64, stride=97, max
         step = len(rows) / max_rows
         rows = [rows[int(j * step)] for j in range(max_rows)]
     return rows
+
+
+# ----------------------------------------------------------------------------- packed variable-length batches
+
+@dataclass(frozen=True)
+class VarlenWorkload:
+    """A packed batch of sequences: q [total_q, H, D], k / v [total_k, H, D].
+
+    Lengths: `lengths` if given, else `nseq` query lengths drawn uniformly from
+    [min_len, max_len] with the workload's seed (key length = query length).
+    Values as for Workload: fp32 standard normals times the std, rounded."""
+    name: str
+    dtype: str
+    H: int
+    D: int
+    causal: bool
+    scale: float
+    nseq: int = 0
+    min_len: int = 1
+    max_len: int = 1
+    lengths: tuple = ()     # ((Sq, Sk), ...) overrides the drawn lengths
+    qk_std: float = 1.0
+    v_std: float = 1.0
+    seed: int = 47
+
+    def seq_lengths(self):
+        if self.lengths:
+            return [tuple(x) for x in self.lengths]
+        g = torch.Generator(device="cpu")
+        g.manual_seed(int(self.seed) + 1000)
+        n = torch.randint(self.min_len, self.max_len + 1, (self.nseq,), generator=g).tolist()
+        return [(a, a) for a in n]
+
+    def offsets(self):
+        """cu_seqlens_q, cu_seqlens_k as int32 CPU tensors of nseq + 1 offsets."""
+        ls = self.seq_lengths()
+        cq = [0]
+        ck = [0]
+        for a, b in ls:
+            cq.append(cq[-1] + a)
+            ck.append(ck[-1] + b)
+        return torch.tensor(cq, dtype=torch.int32), torch.tensor(ck, dtype=torch.int32)
+
+    def flops(self):
+        """Sum over sequences of 4*H*Sq*Sk*D, halved when causal (the dense metric's convention)."""
+        f = sum(4.0 * self.H * a * b * self.D for a, b in self.seq_lengths())
+        return f / 2 if self.causal else f
+
+
+VARLEN_WORKLOADS = {
+    "bf16_varlen_n16_h32_d128_causal": VarlenWorkload(
+        "bf16_varlen_n16_h32_d128_causal", "bf16", 32, 128, True, 1.0 / math.sqrt(128),
+        nseq=16, min_len=128, max_len=8192, seed=47),
+}
+
+
+def make_varlen_qkv(w: VarlenWorkload, device="cpu"):
+    """Draws packed q, k, v (recipe as make_qkv) and returns (q, k, v, cu_q, cu_k)."""
+    cu_q, cu_k = w.offsets()
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(w.seed))
+    dt = DTYPES[w.dtype]
+    tq, tk = int(cu_q[-1]), int(cu_k[-1])
+    q = (torch.randn((tq, w.H, w.D), generator=g, dtype=torch.float32) * w.qk_std).to(dt)
+    k = (torch.randn((tk, w.H, w.D), generator=g, dtype=torch.float32) * w.qk_std).to(dt)
+    v = (torch.randn((tk, w.H, w.D), generator=g, dtype=torch.float32) * w.v_std).to(dt)
+    if device != "cpu":
+        q, k, v, cu_q, cu_k = (t.to(device) for t in (q, k, v, cu_q, cu_k))
+    return q, k, v, cu_q, cu_k

@@ -144,6 +144,39 @@ fa_status fa_fwd_ws(const void *q, const void *k, const void *v, void *o, float 
 size_t fa_fwd_workspace_size(void);
 
 /*
+ * fa_fwd_varlen -- the same forward pass over a batch of B sequences of
+ * different lengths, packed row after row (the uneven-work case of page "64K
+ * long-sequence FlashAttention" (ai6s.net/6a140d07), section "multi-AI-Core
+ * load balancing"; work units of short sequences simply end sooner).
+ * Sequence b owns query rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key /
+ * value rows [cu_seqlens_k[b], cu_seqlens_k[b+1]); it attends only to its own
+ * keys, causal alignment is top-left within the sequence (key j visible to
+ * query i iff j <= i, both counted from the sequence start).
+ *
+ * q, o           [total_q, H, D], fp16 / bf16, contiguous, 16-byte aligned
+ * k, v           [total_k, H, D]
+ * lse            [H, total_q] fp32: lse[h * total_q + row] (natural log)
+ * cu_seqlens_q/k device int32 arrays of B + 1 offsets, non-decreasing, first
+ *                0, last <= total_q / total_k, 4-byte aligned
+ * max_seqlen_q/k upper bounds of the sequence lengths (they size the
+ *                schedule); <= total_q / total_k
+ * workspace      as for fa_fwd_ws, or NULL for the static schedule
+ *
+ * Every other argument is as for fa_fwd.  The offsets live on the device, so
+ * the host cannot check them: a sequence whose offsets are out of range or
+ * decreasing, longer than max_seqlen_q/k, or with queries but no keys, is
+ * skipped (its o and lse rows are not written) and the next
+ * fa_device_status() returns FA_ERR_INVALID_ARG.  Sequences with no query
+ * rows are allowed.  Host-side errors are returned as for fa_fwd.
+ */
+fa_status fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                        const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                        int64_t B, int64_t H, int64_t total_q, int64_t total_k,
+                        int64_t max_seqlen_q, int64_t max_seqlen_k, int64_t D,
+                        int causal, float scale, fa_dtype dtype,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * fa_selftest_wait_timeout -- exercises the kernel's failure detection
  * without a fault.  The kernel is launched as by fa_fwd (same arguments and
  * validation), but its producer warp issues no loads and every wait is limited
@@ -189,8 +222,9 @@ fa_status fa_fwd_noalloc(const void *q, const void *k, const void *v, void *o, f
 /*
  * fa_device_status -- synchronises `stream`, then reads and clears the
  * library's device-side error word on the current device.  Returns FA_OK,
- * FA_ERR_TIMEOUT if a kernel stopped at a wait limit since the last call, or
- * FA_ERR_CUDA if the synchronisation itself failed.
+ * FA_ERR_TIMEOUT if a kernel stopped at a wait limit since the last call,
+ * else FA_ERR_INVALID_ARG if a variable-length batch had invalid sequence
+ * offsets (fa_fwd_varlen), or FA_ERR_CUDA if the synchronisation itself failed.
  */
 fa_status fa_device_status(void *stream);
 

@@ -133,6 +133,44 @@ class Oracle:
             return o.reshape(B, H, Sq, D), lse.reshape(B, H, Sq)
         return o, lse
 
+    def fwd_varlen(self, q, k, v, cu_q, cu_k, *, causal=False, scale=None, rows=None, threads=0):
+        """Attention forward over a packed batch of sequences of different lengths.
+
+        q: [total_q, H, D], k, v: [total_k, H, D]; sequence b owns query rows
+        cu_q[b] .. cu_q[b+1]-1 and key rows cu_k[b] .. cu_k[b+1]-1, and is the
+        standard attention above on its own rows (causal: top-left aligned
+        within the sequence).  This is the dense oracle applied to each
+        sequence as a batch of one, in the packed [S, H, D] = BSND layout; it
+        adds no arithmetic.  Returns (o [total_q, H, D], lse [H, total_q]),
+        fp64; with rows (packed query row ids), o is [n, H, D] and lse [H, n]
+        for those rows only.  A sequence with query rows but no keys raises
+        ValueError (its softmax is over an empty set).
+        """
+        cu_q = [int(x) for x in cu_q]
+        cu_k = [int(x) for x in cu_k]
+        if len(cu_q) != len(cu_k) or len(cu_q) < 2:
+            raise ValueError("cu_q and cu_k must hold the same number (B + 1 >= 2) of offsets")
+        if q.ndim != 3 or k.ndim != 3:
+            raise ValueError("q must be [total_q, H, D] and k, v [total_k, H, D]")
+        total_q, H, D = q.shape
+        want = np.arange(total_q) if rows is None else np.asarray(rows, dtype=np.int64)
+        o = np.zeros((len(want), H, D), dtype=np.float64)
+        lse = np.zeros((H, len(want)), dtype=np.float64)
+        for b in range(len(cu_q) - 1):
+            q0, q1, k0, k1 = cu_q[b], cu_q[b + 1], cu_k[b], cu_k[b + 1]
+            sel = np.nonzero((want >= q0) & (want < q1))[0]   # positions in the output
+            if q1 == q0 or len(sel) == 0:
+                continue
+            if k1 == k0:
+                raise ValueError(f"sequence {b} has query rows but no keys")
+            local = want[sel] - q0
+            flat = (np.arange(H)[:, None] * (q1 - q0) + local[None, :]).reshape(-1)   # (h * Sq_b + i)
+            ob, lb = self.fwd(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], layout="BSND", causal=causal,
+                              scale=scale, rows=flat, threads=threads)
+            o[sel] = ob.reshape(H, len(sel), D).transpose(1, 0, 2)
+            lse[:, sel] = lb.reshape(H, len(sel))
+        return o, lse
+
     def weights(self, q, k, v, *, row, layout="BHSD", causal=False, scale=None):
         """Softmax weights (length Sk, zero where masked) of one flat query row."""
         lay = _LAYOUTS[layout] if isinstance(layout, str) else int(layout)

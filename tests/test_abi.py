@@ -179,3 +179,32 @@ def test_selftest_limit_range_and_argument_checks(lib):
         assert call_selftest(**kw) == call(**kw) == fa.FA_ERR_INVALID_ARG
     assert call_selftest(D=96) == fa.FA_ERR_UNSUPPORTED
     assert call_selftest(Sq=0) == fa.FA_OK
+
+
+CUQ, CUK = 0x70000000, 0x70001000
+
+
+def call_varlen(**kw):
+    a = dict(q=Q, k=K, v=V, o=O, lse=L, cu_q=CUQ, cu_k=CUK, B=3, H=2, total_q=600, total_k=700, max_q=300,
+             max_k=400, D=128, causal=1, scale=0.1, dtype=fa.FA_BF16, ws=None, ws_bytes=0)
+    a.update(kw)
+    return fa.fa_fwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cu_q"], a["cu_k"], a["B"], a["H"],
+                            a["total_q"], a["total_k"], a["max_q"], a["max_k"], a["D"], a["causal"], a["scale"],
+                            a["dtype"], a["ws"], a["ws_bytes"], None)
+
+
+def test_varlen_host_validation(lib):
+    """Checks of the packed entry that return before any device call."""
+    for kw in (dict(B=0), dict(H=0), dict(total_q=-1), dict(max_k=-1), dict(dtype=7), dict(scale=float("inf")),
+               dict(max_q=601), dict(max_k=701), dict(max_k=0), dict(cu_q=0), dict(cu_k=0), dict(lse=0),
+               dict(ws=WS, ws_bytes=4)):
+        assert call_varlen(**kw) == fa.FA_ERR_INVALID_ARG, kw
+    assert call_varlen(D=96) == fa.FA_ERR_UNSUPPORTED
+    assert call_varlen(total_q=0, max_q=0) == fa.FA_OK
+    assert call_varlen(max_q=0) == fa.FA_OK
+    assert call_varlen(cu_q=CUQ + 2) == fa.FA_ERR_MISALIGNED
+    assert call_varlen(q=Q + 8) == fa.FA_ERR_MISALIGNED
+    assert call_varlen(ws=WS + 4, ws_bytes=16) == fa.FA_ERR_MISALIGNED
+    assert call_varlen(o=CUQ) == fa.FA_ERR_ALIAS
+    assert call_varlen(lse=Q + 64) == fa.FA_ERR_ALIAS
+    assert call_varlen(ws=CUK, ws_bytes=16) == fa.FA_ERR_ALIAS
