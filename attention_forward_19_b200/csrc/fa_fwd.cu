@@ -83,10 +83,11 @@ constexpr float HEADROOM_LOG2 = 8.0f;  // bf16 only: a moved reference sits this
 #define FA_EMU_PAIRS 0
 #endif
 // Of the 64 exp2 pairs of a 128-key row, this many (spread evenly) run on the
-// FMA pipe.  The softmax loop is bound by instruction dispatch as much as by
-// MUFU: a MUFU pair costs 1 dispatch slot per value but 8 pipe cycles, an
-// emulated pair about 22 dispatch slots.  Measured on the workloads, 0 to 6
-// of 64 are within noise of each other and more is slower, so the default is 0.
+// FMA pipe.  The softmax loop is bound by latency and instruction dispatch as
+// much as by MUFU: a MUFU pair costs 1 dispatch slot per value but 8 pipe
+// cycles, an emulated pair about 22 dispatch slots.  Measured on the four
+// large workloads (calls of the variants interleaved, sustained clocks), 4 to
+// 10 of 64 are 3-10 % slower than none, so the default is 0.
 constexpr int EMU_PAIRS = FA_EMU_PAIRS;
 __host__ __device__ constexpr bool emulated_pair(int i, int e) { return (i * e) / 64 != ((i + 1) * e) / 64; }
 
@@ -458,15 +459,16 @@ __device__ __forceinline__ uint32_t imad_shl23(uint32_t a, uint32_t b) {
 // 2^r is a polynomial (constant term 1; near-minimax in relative error, fitted
 // by csrc/gen_exp2_poly.py: 1.0e-4 at degree 3, 2.9e-6 at degree 4), and 2^j
 // is added to its exponent field.  x is clamped to [-125, 64] so the exponent
-// stays normal: 2^-125 stands in for anything smaller, and an argument above
-// 64 (only possible on a rejected speculative pass, see the softmax) still
-// gives a large positive value.
+// stays normal: 2^-125 stands in for any finite value below (-inf, a masked
+// key, gives exactly 0), and an argument above 64 (only possible on a
+// rejected speculative pass, see the softmax) still gives a large positive
+// value.
 template <int DEG>
 __device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& y0, float& y1) {
-  float x0, x1;
-  f2unpack(x2, x0, x1);
-  x0 = fminf(fmaxf(x0, -125.f), 64.f);
-  x1 = fminf(fmaxf(x1, -125.f), 64.f);
+  float xin0, xin1;
+  f2unpack(x2, xin0, xin1);
+  const float x0 = fminf(fmaxf(xin0, -125.f), 64.f);
+  const float x1 = fminf(fmaxf(xin1, -125.f), 64.f);
   const uint64_t magic = f2pack(12582912.f, 12582912.f);
   const uint64_t t = fadd2(f2pack(x0, x1), magic);
   const uint64_t neg_j = ffma2(t, f2pack(-1.f, -1.f), magic);
@@ -488,6 +490,9 @@ __device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& y0, float& y1
   // which runs on the FMA pipe); bits(t) * 2^23 keeps only j * 2^23 modulo 2^32
   y0 = __uint_as_float(imad_shl23(__float_as_uint(t0), __float_as_uint(p0)));
   y1 = __uint_as_float(imad_shl23(__float_as_uint(t1), __float_as_uint(p1)));
+  // a masked key (-inf) weighs exactly 0, as MUFU's ex2 gives
+  y0 = xin0 >= -125.f ? y0 : 0.f;
+  y1 = xin1 >= -125.f ? y1 : 0.f;
 }
 
 // max over the row of s * c (c > 0: max(s) * c; c < 0: min(s) * c; c = 0: 0).
@@ -936,8 +941,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float m_prev = m;
         bool exact = (j == 0);
         if (!exact) {
-          rowsum = masked ? exp_pack_row<BF16, 0>(sr, cc, -m_use, pk, p_top)
-                          : exp_pack_row<BF16, EMU_PAIRS>(sr, cc, -m_use, pk, p_top);
+          rowsum = exp_pack_row<BF16, EMU_PAIRS>(sr, cc, -m_use, pk, p_top);
           exact = __any_sync(0xffffffffu, !(p_top <= RESCALE_POW2));
           if (exact) load_s(sr);
         }
@@ -950,8 +954,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // HEADROOM + RESCALE_LOG2 before the next move; fp16 keeps the max.
           if (grow) m = m_cand + (BF16 ? HEADROOM_LOG2 : 0.f);
           m_use = (m == -INFINITY) ? 0.f : m;
-          rowsum = masked ? exp_pack_row<BF16, 0>(sr, cc, -m_use, pk, p_top)
-                          : exp_pack_row<BF16, EMU_PAIRS>(sr, cc, -m_use, pk, p_top);
+          rowsum = exp_pack_row<BF16, EMU_PAIRS>(sr, cc, -m_use, pk, p_top);
         }
 #pragma unroll
         for (int h2 = 0; h2 < BN / 64; ++h2)
