@@ -169,3 +169,12 @@ def make_varlen_qkv(w: VarlenWorkload, device="cpu"):
     if device != "cpu":
         q, k, v, cu_q, cu_k = (t.to(device) for t in (q, k, v, cu_q, cu_k))
     return q, k, v, cu_q, cu_k
+
+
+def make_dout(w: Workload, device="cpu"):
+    """Draws the output gradient dO for workload w: float32 standard normals of
+    q's shape from seed + 500, rounded to the dtype (q, k, v are unchanged)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(w.seed) + 500)
+    do = torch.randn(w.q_shape(), generator=g, dtype=torch.float32).to(DTYPES[w.dtype])
+    return do.to(device) if device != "cpu" else do

@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for the attention forward pass.
+"""fp64 CPU oracle for the attention forward pass (attn, attn_oracle.c) and its
+backward (attn_bwd).
 
 TEST INFRASTRUCTURE, NOT PRODUCT CODE: only the test suite, the package smoke
 check and the benchmark's CPU-baseline / reference arm may import it.  It
