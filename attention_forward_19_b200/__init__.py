@@ -36,7 +36,8 @@ FA_BF16 = 1
 LAYOUTS = {"BSND": FA_BSND, "BHSD": FA_BHSD}
 
 # Names every public symbol of include/fa_fwd.h.
-EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_noalloc", "fa_fwd_varlen",
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_noalloc", "fa_fwd_varlen", "fa_bwd",
+                    "fa_bwd_workspace_size",
                     "fa_selftest_wait_timeout", "fa_device_status", "fa_query_support", "fa_status_string",
                     "fa_last_cuda_error", "fa_version")
 
@@ -83,6 +84,11 @@ def load_library(path=None, rebuild_if_stale=True):
     lib.fa_fwd_varlen.restype = c_int
     lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, c_int, c_float,
                                   c_int, vp, ctypes.c_size_t, vp]
+    lib.fa_bwd.restype = c_int
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int,
+                           vp, ctypes.c_size_t, vp]
+    lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.fa_bwd_workspace_size.argtypes = [i64, i64, i64]
     lib.fa_selftest_wait_timeout.restype = c_int
     lib.fa_selftest_wait_timeout.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float,
                                              c_int, ctypes.c_uint32, vp]
@@ -135,6 +141,18 @@ def fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, H, total_q, total_k, max_q, ma
     return lib.fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, int(B), int(H), int(total_q), int(total_k), int(max_q),
                              int(max_k), int(D), int(bool(causal)), float(scale), int(dtype), workspace,
                              int(workspace_bytes), stream)
+
+
+def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, Sq, Sk, D, layout, causal, scale, dtype, workspace,
+           workspace_bytes, stream):
+    """The C fa_bwd (gradients) with raw pointers and sizes; returns the fa_status code."""
+    lib = load_library()
+    return lib.fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
+                      int(bool(causal)), float(scale), int(dtype), workspace, int(workspace_bytes), stream)
+
+
+def fa_bwd_workspace_size(B, H, Sq):
+    return load_library().fa_bwd_workspace_size(int(B), int(H), int(Sq))
 
 
 def fa_selftest_wait_timeout(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, wait_limit_us,
@@ -321,6 +339,50 @@ def flash_attention_varlen_forward(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seql
     if st != FA_OK:
         raise FaError(st, "fa_fwd_varlen")
     return out, lse
+
+
+def flash_attention_backward(q, k, v, o, lse, dout, layout="BSND", causal=False, scale=None, dq=None, dk=None,
+                             dv=None, stream=None, workspace=None):
+    """Gradients (dq, dk, dv) of flash_attention_forward through the C ABI.
+
+    q, k, v as for the forward; o and lse as the forward returned them; dout
+    (dL/dO) like o.  Returns (dq, dk, dv) shaped like q, k, v.  `workspace`, a
+    uint8 CUDA tensor of fa_bwd_workspace_size(B, H, Sq) bytes, is allocated
+    here when not given.  Runs on `stream` without synchronising.
+    """
+    import torch
+    lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    B, H, Sq, Sk, D = _dims(q, k, lay)
+    for name, t, like in (("v", v, k), ("o", o, q), ("dout", dout, q)):
+        if t.shape != like.shape or t.dtype != q.dtype or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous tensor of shape {tuple(like.shape)} and q's dtype")
+    for name, t in (("q", q), ("k", k)):
+        if not t.is_contiguous() or t.dtype != q.dtype:
+            raise ValueError(f"{name} must be contiguous and share q's dtype")
+    if lse.shape != (B, H, Sq) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be the forward's contiguous fp32 [B, H, Sq] tensor")
+    dt = _dtype_code(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t, like in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        if t.shape != like.shape or t.dtype != like.dtype or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous tensor like {name[1:]}")
+    nbytes = fa_bwd_workspace_size(B, H, Sq)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device) if q.is_cuda else None
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, Sq, Sk, D, lay, causal, scale, dt,
+                workspace.data_ptr(), wbytes, sptr)
+    if st != FA_OK:
+        raise FaError(st, "fa_bwd")
+    return dq, dk, dv
 
 
 def check_device_status(stream=None):

@@ -9,6 +9,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "fa_fwd.cu")
+DEPS = [os.path.join(PKG, "csrc", "fa_bwd_impl.cuh")]   # included by fa_fwd.cu
 HDR = os.path.join(ROOT, "include", "fa_fwd.h")
 LIB = os.path.join(PKG, "libfa_fwd.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -23,7 +24,7 @@ def _stale(out, sources):
 
 def build(force=False, verbose=False, out=LIB):
     """Compiles fa_fwd.cu when the library is missing or older than its sources; returns its path."""
-    if not force and not _stale(out, [SRC, HDR]):
+    if not force and not _stale(out, [SRC, HDR] + DEPS):
         return out
     cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
            "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"),

@@ -1545,3 +1545,6 @@ int fa_last_cuda_error(void) { return t_last_cuda_error; }
 int fa_version(void) { return FA_VERSION; }
 
 }  // extern "C"
+
+// The backward pass (gradients) shares this translation unit's helpers.
+#include "fa_bwd_impl.cuh"

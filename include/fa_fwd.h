@@ -177,6 +177,34 @@ fa_status fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, fl
                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * fa_bwd -- gradients of the forward pass: given q, k, v, the forward's o and
+ * lse, and dout = dL/dO, writes dq, dk, dv (same shapes, layout and dtype as
+ * q, k, v).  The weights are recomputed from q, k and lse (page "FlashAttention
+ * in ops-transformer on Ascend NPU" (ai6s.net/6a0d3bfb), section "how FA runs
+ * on the NPU": recomputation), then dV = P^T dO, dS = P * (dO V^T -
+ * rowsum(dO * O)), dQ = scale dS K, dK = scale dS^T Q, with the forward's
+ * causal mask.  Deterministic: every gradient row is accumulated by one CTA in
+ * a fixed order, with no atomics (page "catlass FlashAttention template
+ * tuning" (hwcomputing.csdn.net/6a0d4681): the backward's `deterministic`
+ * switch).  fp32 accumulation; results rounded to the input dtype.
+ *
+ * q, k, v, o, dout, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, stream
+ *                  as for fa_fwd (o and lse as fa_fwd wrote them)
+ * dq, dk, dv       outputs, caller-owned, 16-byte aligned, fully overwritten
+ * workspace        device memory of fa_bwd_workspace_size(B, H, Sq) bytes,
+ *                  16-byte aligned, caller-owned scratch (per-row sums)
+ *
+ * Errors as for fa_fwd; the outputs and the workspace must not overlap each
+ * other or any input (FA_ERR_ALIAS).  Sq = 0 sets dk = dv = 0.
+ */
+size_t fa_bwd_workspace_size(int64_t B, int64_t H, int64_t Sq);
+fa_status fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                 const float *lse, void *dq, void *dk, void *dv,
+                 int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D,
+                 fa_layout layout, int causal, float scale, fa_dtype dtype,
+                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * fa_selftest_wait_timeout -- exercises the kernel's failure detection
  * without a fault.  The kernel is launched as by fa_fwd (same arguments and
  * validation), but its producer warp issues no loads and every wait is limited

@@ -208,3 +208,34 @@ def test_varlen_host_validation(lib):
     assert call_varlen(o=CUQ) == fa.FA_ERR_ALIAS
     assert call_varlen(lse=Q + 64) == fa.FA_ERR_ALIAS
     assert call_varlen(ws=CUK, ws_bytes=16) == fa.FA_ERR_ALIAS
+
+
+DQ, DK, DV, DO_, WSB = 0x71000000, 0x72000000, 0x73000000, 0x74000000, 0x75000000
+
+
+def call_bwd(**kw):
+    a = dict(q=Q, k=K, v=V, o=O, dout=DO_, lse=L, dq=DQ, dk=DK, dv=DV, B=1, H=2, Sq=512, Sk=512, D=128,
+             layout=fa.FA_BHSD, causal=1, scale=0.1, dtype=fa.FA_BF16, ws=WSB, ws_bytes=1 << 20)
+    a.update(kw)
+    return fa.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["dout"], a["lse"], a["dq"], a["dk"], a["dv"], a["B"], a["H"],
+                     a["Sq"], a["Sk"], a["D"], a["layout"], a["causal"], a["scale"], a["dtype"], a["ws"],
+                     a["ws_bytes"], None)
+
+
+def test_bwd_workspace_size():
+    assert fa.fa_bwd_workspace_size(1, 2, 512) == 2 * 2 * 512 * 4
+    assert fa.fa_bwd_workspace_size(1, 2, 513) == 2 * 2 * 640 * 4     # each head padded to whole 128-row tiles
+    assert fa.fa_bwd_workspace_size(0, 2, 512) == 0
+
+
+def test_bwd_host_validation(lib):
+    for kw in (dict(B=0), dict(Sk=0), dict(layout=5), dict(dtype=9), dict(scale=float("nan")), dict(q=0),
+               dict(lse=0), dict(dq=0), dict(ws=0), dict(ws_bytes=100)):
+        assert call_bwd(**kw) == fa.FA_ERR_INVALID_ARG, kw
+    assert call_bwd(D=80) == fa.FA_ERR_UNSUPPORTED
+    assert call_bwd(dq=DQ + 8) == fa.FA_ERR_MISALIGNED
+    assert call_bwd(ws=WSB + 4) == fa.FA_ERR_MISALIGNED
+    assert call_bwd(lse=L + 2) == fa.FA_ERR_MISALIGNED
+    assert call_bwd(dq=Q) == fa.FA_ERR_ALIAS
+    assert call_bwd(dk=DV) == fa.FA_ERR_ALIAS
+    assert call_bwd(ws=DO_) == fa.FA_ERR_ALIAS
