@@ -18,20 +18,24 @@
 //      (each head padded to whole 128-row tiles, padding +inf / 0).
 //   2. dK/dV kernel, one CTA per 128-key tile: S^T = K Q_i^T and
 //      dP^T = V dO_i^T for every visible query tile i put the keys on the TMEM
-//      lanes; one thread per key computes P^T and dS^T, writes them (16-bit)
-//      over S^T / dP^T, and dV += P^T dO_i, dK += dS^T Q_i take them as the
-//      TMEM operand -- the same MMA forms as the forward's O += P V.
+//      lanes; two threads per key (one per half of the query columns) compute
+//      P^T and dS^T, write them (16-bit) over S^T / dP^T, and dV += P^T dO_i,
+//      dK += dS^T Q_i take them as the TMEM operand -- the same MMA forms as
+//      the forward's O += P V.
 //   3. dQ kernel, one CTA per 128-query tile: S = Q K_j^T, dP = dO V_j^T,
-//      one thread per query row computes dS, and dQ += dS K_j.
+//      two threads per query row compute dS, and dQ += dS K_j.
 // S and dP are computed by both kernels (7 tile products instead of 5): the
 // price of having every gradient row owned by exactly one CTA.
 
 namespace fa {
 namespace bwd {
 
-constexpr int THREADS = 192;   // warps 0-3 compute (one thread per tile row), 4 load, 5 MMA
-constexpr int LOAD_WARP = 4;
-constexpr int MMA_WARP = 5;
+// Warps 0-7: two compute warpgroups on the same tile (warps w and w + 4 read
+// the same TMEM lanes, one row each; group g takes columns [64 g, 64 g + 64)).
+// Warp 8: loads.  Warp 9: MMA.
+constexpr int THREADS = 320;
+constexpr int LOAD_WARP = 8;
+constexpr int MMA_WARP = 9;
 constexpr int NSTAGE = 2;      // streamed tile pairs in flight
 
 template <int D>
@@ -42,8 +46,9 @@ struct Cfg {
   static constexpr int ST_FULL = 1;            // a streamed stage (two tiles, + two vectors for dK/dV)
   static constexpr int ST_EMPTY = ST_FULL + NSTAGE;
   static constexpr int S_FULL = ST_EMPTY + NSTAGE;   // S and dP of this step are in TMEM
-  static constexpr int P_FULL = S_FULL + 1;          // the 16-bit operands are written (128 arrivals)
-  static constexpr int ACC_FULL = P_FULL + 1;        // the accumulators are final
+  static constexpr int P_FULL = S_FULL + 1;          // the 16-bit operands are written (256 arrivals)
+  static constexpr int RD_DONE = P_FULL + 1;         // both groups have read S and dP (256 arrivals)
+  static constexpr int ACC_FULL = RD_DONE + 1;       // the accumulators are final
   static constexpr int DRAIN = ACC_FULL + 1;
   static constexpr int NBAR = DRAIN + 1;
   static constexpr int SMEM_FIX = 0;
@@ -168,7 +173,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bar(C::ST_EMPTY + s), 1);
     }
     mbar_init(bar(C::S_FULL), 1);
-    mbar_init(bar(C::P_FULL), BM);
+    mbar_init(bar(C::P_FULL), 2 * BM);
+    mbar_init(bar(C::RD_DONE), 2 * BM);
     mbar_init(bar(C::ACC_FULL), 1);
     mbar_init(bar(C::DRAIN), 1);
     *abort_flag = 0;
@@ -259,9 +265,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- compute warpgroup: one thread per key
-    const int rit = warp * 32 + lane;
+    const int quad = warp & 3, grp = warp >> 2;
+    const int rit = quad * 32 + lane;
     const int key = k0 + rit;
-    const uint32_t lane_bits = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_bits = (uint32_t)(quad * 32) << 16;
     const uint32_t tST = tmem + lane_bits, tDPT = tmem + lane_bits + BM;
     const uint32_t tDV = tmem + lane_bits + 2 * BM, tDK = tmem + lane_bits + 2 * BM + D;
     const float c = p.scale_log2;
@@ -281,20 +288,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       // causal: query q sees this key iff q >= key; only tiles that reach
       // below the key need the test
       const bool masked = p.causal && (q0 < k0 + BM - 1);
+      uint32_t pp[32], pd[32];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t s[64], dp[64];
-        tmem_ld32(tST + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        tmem_ld32(tST + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-        tmem_ld32(tDPT + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-        tmem_ld32(tDPT + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+      for (int ch = 0; ch < 2; ++ch) {
+        const int col = grp * 64 + ch * 32;          // query columns [col, col + 32)
+        uint32_t s[32], dp[32];
+        tmem_ld32(tST + col, s);
+        tmem_ld32(tDPT + col, dp);
         tmem_wait_ld();
         reg_fence(s);
         reg_fence(dp);
-        uint32_t pp[32], pd[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int qa = hh * 64 + 2 * e;     // query column within the tile
+        for (int e = 0; e < 16; ++e) {
+          const int qa = col + 2 * e;
           const float4 l4 = *reinterpret_cast<const float4*>(vl + (qa & ~3));
           const float4 d4 = *reinterpret_cast<const float4*>(vd + (qa & ~3));
           const float la = (qa & 2) ? l4.z : l4.x, lb = (qa & 2) ? l4.w : l4.y;
@@ -307,13 +313,19 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           const float ga = pa * (__uint_as_float(dp[2 * e]) - da);
           const float gb = pb * (__uint_as_float(dp[2 * e + 1]) - db);
-          pp[e] = pack2<BF16>(pa, pb);
-          pd[e] = pack2<BF16>(ga, gb);
+          pp[ch * 16 + e] = pack2<BF16>(pa, pb);
+          pd[ch * 16 + e] = pack2<BF16>(ga, gb);
         }
-        // P^T over S^T columns [32 hh, 32 hh + 32), dS^T over dP^T's (already read)
-        tmem_st32(tST + hh * 32, pp);
-        tmem_st32(tDPT + hh * 32, pd);
       }
+      // P^T / dS^T of group g go over S^T / dP^T columns [32 g, 32 g + 32),
+      // which group 0 reads: both groups finish reading first.
+      tc_fence_before();
+      mbar_arrive(bar(C::RD_DONE));
+      ok = wait_bar(bar(C::RD_DONE), n & 1u, abort_flag, limit);
+      if (!ok) break;
+      tc_fence_after();
+      tmem_st32(tST + grp * 32, pp);
+      tmem_st32(tDPT + grp * 32, pd);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::P_FULL));
@@ -322,24 +334,21 @@ __global__ void __launch_bounds__(THREADS, 1)
     const bool store = key < p.Sk;
     uint8_t* dvrow = p.dv + (size_t)b * p.k_bs + (size_t)h * p.k_hs + (size_t)key * p.k_rs;
     uint8_t* dkrow = p.dk + (size_t)b * p.k_bs + (size_t)h * p.k_hs + (size_t)key * p.k_rs;
+    // group 0 stores the dV row, group 1 the dK row
+    uint8_t* dst = grp ? dkrow : dvrow;
     if (nq == 0) {
       // no query sees this key: its gradients are zero
       if (store) {
 #pragma unroll
-        for (int e = 0; e < D * 2 / 16; ++e) {
-          reinterpret_cast<uint4*>(dvrow)[e] = make_uint4(0, 0, 0, 0);
-          reinterpret_cast<uint4*>(dkrow)[e] = make_uint4(0, 0, 0, 0);
-        }
+        for (int e = 0; e < D * 2 / 16; ++e) reinterpret_cast<uint4*>(dst)[e] = make_uint4(0, 0, 0, 0);
       }
     } else if (ok) {
       ok = wait_bar(bar(C::ACC_FULL), 0, abort_flag, limit);
       if (ok) {
         tc_fence_after();
-#pragma unroll
-        for (int which = 0; which < 2; ++which) {
-          const uint32_t src = which ? tDK : tDV;
-          uint8_t* dst = which ? dkrow : dvrow;
-          const float f = which ? p.scale : 1.f;
+        {
+          const uint32_t src = grp ? tDK : tDV;
+          const float f = grp ? p.scale : 1.f;
 #pragma unroll
           for (int q4 = 0; q4 < D / 32; ++q4) {
             uint32_t r[32];
@@ -407,7 +416,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bar(C::ST_EMPTY + s), 1);
     }
     mbar_init(bar(C::S_FULL), 1);
-    mbar_init(bar(C::P_FULL), BM);
+    mbar_init(bar(C::P_FULL), 2 * BM);
+    mbar_init(bar(C::RD_DONE), 2 * BM);
     mbar_init(bar(C::ACC_FULL), 1);
     mbar_init(bar(C::DRAIN), 1);
     *abort_flag = 0;
@@ -486,9 +496,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- compute warpgroup: one thread per query row
-    const int rit = warp * 32 + lane;
+    const int quad = warp & 3, grp = warp >> 2;
+    const int rit = quad * 32 + lane;
     const int row = q0 + rit;
-    const uint32_t lane_bits = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_bits = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + lane_bits, tDP = tmem + lane_bits + BN, tDQ = tmem + lane_bits + 2 * BN;
     const float c = p.scale_log2;
     const size_t vo = (size_t)bh * p.Sq_pad + (size_t)row;     // padded: in bounds for every row of the tile
@@ -503,30 +514,37 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool masked = (c0 + BN > p.Sk) || (p.causal && c0 + BN - 1 > q0);
       int lim = p.Sk - 1 - c0;                 // last key (relative) this row sees
       if (p.causal) lim = min(lim, row - c0);
+      uint32_t pd[32];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t s[64], dp[64];
-        tmem_ld32(tS + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-        tmem_ld32(tS + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-        tmem_ld32(tDP + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-        tmem_ld32(tDP + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+      for (int ch = 0; ch < 2; ++ch) {
+        const int col = grp * 64 + ch * 32;    // key columns [col, col + 32)
+        uint32_t s[32], dp[32];
+        tmem_ld32(tS + col, s);
+        tmem_ld32(tDP + col, dp);
         tmem_wait_ld();
         reg_fence(s);
         reg_fence(dp);
-        uint32_t pd[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int ka = hh * 64 + 2 * e;
+        for (int e = 0; e < 16; ++e) {
+          const int ka = col + 2 * e;
           float pa = ex2(fmaf(__uint_as_float(s[2 * e]), c, -lse2));
           float pb = ex2(fmaf(__uint_as_float(s[2 * e + 1]), c, -lse2));
           if (masked) {
             if (ka > lim) pa = 0.f;
             if (ka + 1 > lim) pb = 0.f;
           }
-          pd[e] = pack2<BF16>(pa * (__uint_as_float(dp[2 * e]) - dsum), pb * (__uint_as_float(dp[2 * e + 1]) - dsum));
+          pd[ch * 16 + e] = pack2<BF16>(pa * (__uint_as_float(dp[2 * e]) - dsum),
+                                        pb * (__uint_as_float(dp[2 * e + 1]) - dsum));
         }
-        tmem_st32(tS + hh * 32, pd);   // dS over S columns [32 hh, 32 hh + 32) (already read)
       }
+      // dS of group g goes over S columns [32 g, 32 g + 32), which group 0
+      // reads: both groups finish reading first.
+      tc_fence_before();
+      mbar_arrive(bar(C::RD_DONE));
+      ok = wait_bar(bar(C::RD_DONE), (uint32_t)j & 1u, abort_flag, limit);
+      if (!ok) break;
+      tc_fence_after();
+      tmem_st32(tS + grp * 32, pd);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::P_FULL));
@@ -535,8 +553,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (ok) {
       tc_fence_after();
       uint8_t* dqrow = p.dq + (size_t)b * p.q_bs + (size_t)h * p.q_hs + (size_t)row * p.q_rs;
+      // group g stores dQ columns [g D/2, (g + 1) D/2)
 #pragma unroll
-      for (int q4 = 0; q4 < D / 32; ++q4) {
+      for (int q2 = 0; q2 < D / 64; ++q2) {
+        const int q4 = grp * (D / 64) + q2;
         uint32_t r[32];
         tmem_ld32(tDQ + q4 * 32, r);
         tmem_wait_ld();

@@ -14,6 +14,11 @@ are larger than the 126 MB L2, so no flush is done between steps.
 
 --impl reference runs the fp64 CPU oracle (the parity reference) on rank 0
 on a bounded row sample of the same workload, each step one sample.
+
+--backward times the backward pass (fa_bwd: dq, dk, dv from the forward's o
+and lse) on the same workload instead, and prints its own JSON line; its
+metric counts 2.5x the forward's flops (five tile products to the forward's
+two, the usual convention), kernel time only.
 """
 import argparse
 import hashlib
@@ -31,7 +36,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from fa_inputs import BENCH_WORKLOAD, WORKLOADS, make_qkv  # noqa: E402
+from fa_inputs import BENCH_WORKLOAD, WORKLOADS, make_dout, make_qkv  # noqa: E402
 
 METRIC = "attn fwd TFLOP/s (causal-halved) and % of B200 dense fp16/bf16 tensor peak"
 UNIT = "TFLOP/s"
@@ -312,6 +317,71 @@ def run_native(args, rank, world, local_rank):
     return line
 
 
+def run_backward(args, rank, world, local_rank):
+    """Times the backward pass on the workload (kernel time; one JSON line)."""
+    import attention_forward_19_b200 as fa
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w0 = bench_workload(args)
+    w = rank_workload(w0, rank)
+    q, k, v = make_qkv(w, device=dev)
+    do = make_dout(w, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    o, lse = fa.flash_attention_forward(q, k, v, layout=w.layout, causal=w.causal, scale=w.scale, stream=stream)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(16, fa.fa_bwd_workspace_size(w.B, w.H, w.Sq)), dtype=torch.uint8, device=dev)
+
+    def step():
+        fa.flash_attention_backward(q, k, v, o, lse, do, layout=w.layout, causal=w.causal, scale=w.scale, dq=dq,
+                                    dk=dk, dv=dv, stream=stream, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    fa.check_device_status(stream)
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(cvd.split(",")[local_rank].strip() if cvd else str(local_rank))
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    fa.check_device_status(stream)
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ms_step = ms_total / args.steps
+    flops = 2.5 * w.flops()
+    value = world * flops * args.steps / (ms_total * 1e-3) / 1e12
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (ms_step * 1e-3) / 1e12
+    return {
+        "metric": "attn bwd TFLOP/s (2.5x the causal-halved forward flops)", "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": workload_config(w0, world),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                     "traffic": None,
+                     "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
+                                    if peak_kind == "measured" else "fallback 1590 TFLOP/s",
+                     "algorithmic_flops_per_step": flops,
+                     "note": "the pass computes S and dP twice (7 tile products), the metric counts 5"},
+        "gpu_launches": 3 * args.steps,
+        "gpu_launches_note": "per step: prep, dK/dV and dQ kernels",
+        "clocks": clk,
+    }
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 
@@ -355,6 +425,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="time the kernel only (profiling runs)")
     ap.add_argument("--workload", choices=list(WORKLOADS), default=BENCH_WORKLOAD)
     ap.add_argument("--bh", default=None, help="override B,H of the workload (profiling runs)")
+    ap.add_argument("--backward", action="store_true", help="time the backward pass instead (its own JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -371,7 +442,7 @@ def main():
             torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                                  device_id=torch.device("cuda", local_rank))
         try:
-            line = run_native(args, rank, world, local_rank)
+            line = (run_backward if args.backward else run_native)(args, rank, world, local_rank)
         finally:
             if world > 1:
                 torch.distributed.destroy_process_group()
