@@ -45,10 +45,13 @@ struct Cfg {
   static constexpr int IN_FULL = 0;            // the CTA's two fixed tiles
   static constexpr int ST_FULL = 1;            // a streamed stage (two tiles, + two vectors for dK/dV)
   static constexpr int ST_EMPTY = ST_FULL + NSTAGE;
-  static constexpr int S_FULL = ST_EMPTY + NSTAGE;   // S and dP of this step are in TMEM
-  static constexpr int P_FULL = S_FULL + 1;          // the 16-bit operands are written (256 arrivals)
-  static constexpr int RD_DONE = P_FULL + 1;         // both groups have read S and dP (256 arrivals)
-  static constexpr int ACC_FULL = RD_DONE + 1;       // the accumulators are final
+  static constexpr int S_FULL = ST_EMPTY + NSTAGE;   // S^T (dK/dV) or S and dP (dQ) of a step are in TMEM
+  static constexpr int DP_FULL = S_FULL + 1;         // dP^T of a step is in TMEM (dK/dV)
+  static constexpr int RD_A = DP_FULL + 1;           // both groups have read S^T (dK/dV) or S, dP (dQ): 256 arrivals
+  static constexpr int RD_B = RD_A + 1;              // both groups have read dP^T (dK/dV): 256
+  static constexpr int W_A = RD_B + 1;               // P^T (dK/dV) or dS (dQ) written: 256
+  static constexpr int W_B = W_A + 1;                // dS^T written (dK/dV): 256
+  static constexpr int ACC_FULL = W_B + 1;           // the accumulators are final
   static constexpr int DRAIN = ACC_FULL + 1;
   static constexpr int NBAR = DRAIN + 1;
   static constexpr int SMEM_FIX = 0;
@@ -173,8 +176,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bar(C::ST_EMPTY + s), 1);
     }
     mbar_init(bar(C::S_FULL), 1);
-    mbar_init(bar(C::P_FULL), 2 * BM);
-    mbar_init(bar(C::RD_DONE), 2 * BM);
+    mbar_init(bar(C::DP_FULL), 1);
+    mbar_init(bar(C::RD_A), 2 * BM);
+    mbar_init(bar(C::RD_B), 2 * BM);
+    mbar_init(bar(C::W_A), 2 * BM);
+    mbar_init(bar(C::W_B), 2 * BM);
     mbar_init(bar(C::ACC_FULL), 1);
     mbar_init(bar(C::DRAIN), 1);
     *abort_flag = 0;
@@ -226,37 +232,65 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint64_t dStrMN = sdesc(sStr, BOX_BYTES, 1024);  // MN-major view
       constexpr uint32_t TILE16 = C::TILE >> 4;
       const uint32_t tST = tmem, tDPT = tmem + BM, tDV = tmem + 2 * BM, tDK = tmem + 2 * BM + D;
-      uint32_t n = 0;
-      for (int i = i_begin; i < i_end && ok; ++i, ++n) {
-        const uint32_t st = n % NSTAGE;
-        ok = wait_bar(bar(C::ST_FULL + st), (n / NSTAGE) & 1u, abort_flag, limit);
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t q_k = dStr + (uint64_t)(st * 2 * TILE16);
-        const uint64_t do_k = q_k + TILE16;
+      auto st_products = [&](uint32_t n) {     // S^T(n) = K Q_n^T
+        const uint64_t q_k = dStr + (uint64_t)((n % NSTAGE) * 2 * TILE16);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {   // S^T = K Q_i^T
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
           mma_ss_elect(tST, dK0 + off, q_k + off, IDESC_ST, kk > 0 ? 1u : 0u);
         }
+      };
+      auto dpt_products = [&](uint32_t n) {    // dP^T(n) = V dO_n^T
+        const uint64_t do_k = dStr + (uint64_t)((n % NSTAGE) * 2 * TILE16 + TILE16);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {   // dP^T = V dO_i^T
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
           mma_ss_elect(tDPT, dV0k + off, do_k + off, IDESC_ST, kk > 0 ? 1u : 0u);
         }
-        tc_commit_elect(bar(C::S_FULL));
-        ok = wait_bar(bar(C::P_FULL), n & 1u, abort_flag, limit);
-        if (!ok) break;
+      };
+      // Order of the tensor work: S^T(0), dP^T(0), then per step n
+      //   dV(n), S^T(n+1), dK(n), dP^T(n+1)
+      // so that the compute warps work out P^T(n+1) from S^T(n+1) while
+      // dK(n) and dP^T(n+1) run, and dS^T(n+1) while dV(n+1) and S^T(n+2) run.
+      // S^T(n+1) overwrites P^T(n) and dP^T(n+1) overwrites dS^T(n) only
+      // after the products that read them (tcgen05 MMAs run in issue order).
+      if (ok) ok = wait_bar(bar(C::ST_FULL), 0, abort_flag, limit);
+      if (ok) {
         tc_fence_after();
+        st_products(0);
+        tc_commit_elect(bar(C::S_FULL));
+        dpt_products(0);
+        tc_commit_elect(bar(C::DP_FULL));
+      }
+      for (uint32_t n = 0; n < (uint32_t)nq && ok; ++n) {
+        const uint32_t st = n % NSTAGE;
         const uint64_t q_mn = dStrMN + (uint64_t)(st * 2 * TILE16);
         const uint64_t do_mn = q_mn + TILE16;
+        ok = wait_bar(bar(C::W_A), n & 1u, abort_flag, limit);     // P^T(n) written
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)    // dV += P^T dO_i  (P^T: 8 packed columns per 16 queries)
+        for (int kk = 0; kk < BM / 16; ++kk)    // dV += P^T dO_n  (P^T: 8 packed columns per 16 queries)
           mma_ts_elect(tDV, tST + kk * 8, do_mn + (uint64_t)(kk * 128), IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
+        const bool more = n + 1 < (uint32_t)nq;
+        if (more) {
+          ok = wait_bar(bar(C::ST_FULL + (n + 1) % NSTAGE), ((n + 1) / NSTAGE) & 1u, abort_flag, limit);
+          if (!ok) break;
+          tc_fence_after();
+          st_products(n + 1);
+          tc_commit_elect(bar(C::S_FULL));
+        }
+        ok = wait_bar(bar(C::W_B), n & 1u, abort_flag, limit);     // dS^T(n) written
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)    // dK += dS^T Q_i
+        for (int kk = 0; kk < BM / 16; ++kk)    // dK += dS^T Q_n
           mma_ts_elect(tDK, tDPT + kk * 8, q_mn + (uint64_t)(kk * 128), IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
         tc_commit_elect(bar(C::ST_EMPTY + st));
+        if (more) {
+          dpt_products(n + 1);
+          tc_commit_elect(bar(C::DP_FULL));
+        }
       }
       if (ok) tc_commit_elect(bar(C::ACC_FULL));
       tc_commit_elect(bar(C::DRAIN));
@@ -276,10 +310,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t n = 0;
     for (int i = i_begin; i < i_end && ok; ++i, ++n) {
       const uint32_t st = n % NSTAGE;
-      ok = wait_bar(bar(C::S_FULL), n & 1u, abort_flag, limit);
-      if (!ok) break;
-      tc_fence_after();
-      // the stage's vectors came by a bulk copy: observe its completion too
+      // the stage's query vectors came by a bulk copy: observe its completion
       ok = wait_bar(bar(C::ST_FULL + st), (n / NSTAGE) & 1u, abort_flag, limit);
       if (!ok) break;
       const float* vl = sVec + st * 2 * BM;        // lse2 of the tile's queries
@@ -288,47 +319,75 @@ __global__ void __launch_bounds__(THREADS, 1)
       // causal: query q sees this key iff q >= key; only tiles that reach
       // below the key need the test
       const bool masked = p.causal && (q0 < k0 + BM - 1);
-      uint32_t pp[32], pd[32];
+      // ---- phase A: P^T = 2^(s c - lse2) from S^T (kept in fp32 for phase B)
+      ok = wait_bar(bar(C::S_FULL), n & 1u, abort_flag, limit);
+      if (!ok) break;
+      tc_fence_after();
+      float pr[64];
+      uint32_t pk[32];
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         const int col = grp * 64 + ch * 32;          // query columns [col, col + 32)
-        uint32_t s[32], dp[32];
-        tmem_ld32(tST + col, s);
-        tmem_ld32(tDPT + col, dp);
+        uint32_t sv[32];
+        tmem_ld32(tST + col, sv);
         tmem_wait_ld();
-        reg_fence(s);
-        reg_fence(dp);
+        reg_fence(sv);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int qa = col + 2 * e;
           const float4 l4 = *reinterpret_cast<const float4*>(vl + (qa & ~3));
-          const float4 d4 = *reinterpret_cast<const float4*>(vd + (qa & ~3));
           const float la = (qa & 2) ? l4.z : l4.x, lb = (qa & 2) ? l4.w : l4.y;
-          const float da = (qa & 2) ? d4.z : d4.x, db = (qa & 2) ? d4.w : d4.y;
-          float pa = ex2(fmaf(__uint_as_float(s[2 * e]), c, -la));
-          float pb = ex2(fmaf(__uint_as_float(s[2 * e + 1]), c, -lb));
+          float pa = ex2(fmaf(__uint_as_float(sv[2 * e]), c, -la));
+          float pb = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, -lb));
           if (masked) {
             if (q0 + qa < key) pa = 0.f;
             if (q0 + qa + 1 < key) pb = 0.f;
           }
-          const float ga = pa * (__uint_as_float(dp[2 * e]) - da);
-          const float gb = pb * (__uint_as_float(dp[2 * e + 1]) - db);
-          pp[ch * 16 + e] = pack2<BF16>(pa, pb);
-          pd[ch * 16 + e] = pack2<BF16>(ga, gb);
+          pr[ch * 32 + 2 * e] = pa;
+          pr[ch * 32 + 2 * e + 1] = pb;
+          pk[ch * 16 + e] = pack2<BF16>(pa, pb);
         }
       }
-      // P^T / dS^T of group g go over S^T / dP^T columns [32 g, 32 g + 32),
-      // which group 0 reads: both groups finish reading first.
+      // P^T of group g goes over S^T columns [32 g, 32 g + 32), which group 0
+      // reads: both groups finish reading first.
       tc_fence_before();
-      mbar_arrive(bar(C::RD_DONE));
-      ok = wait_bar(bar(C::RD_DONE), n & 1u, abort_flag, limit);
+      mbar_arrive(bar(C::RD_A));
+      ok = wait_bar(bar(C::RD_A), n & 1u, abort_flag, limit);
       if (!ok) break;
       tc_fence_after();
-      tmem_st32(tST + grp * 32, pp);
-      tmem_st32(tDPT + grp * 32, pd);
+      tmem_st32(tST + grp * 32, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(C::P_FULL));
+      mbar_arrive(bar(C::W_A));
+      // ---- phase B: dS^T = P^T (dP^T - D)
+      ok = wait_bar(bar(C::DP_FULL), n & 1u, abort_flag, limit);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        const int col = grp * 64 + ch * 32;
+        uint32_t dp[32];
+        tmem_ld32(tDPT + col, dp);
+        tmem_wait_ld();
+        reg_fence(dp);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int qa = col + 2 * e;
+          const float4 d4 = *reinterpret_cast<const float4*>(vd + (qa & ~3));
+          const float da = (qa & 2) ? d4.z : d4.x, db = (qa & 2) ? d4.w : d4.y;
+          pk[ch * 16 + e] = pack2<BF16>(pr[ch * 32 + 2 * e] * (__uint_as_float(dp[2 * e]) - da),
+                                        pr[ch * 32 + 2 * e + 1] * (__uint_as_float(dp[2 * e + 1]) - db));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::RD_B));
+      ok = wait_bar(bar(C::RD_B), n & 1u, abort_flag, limit);
+      if (!ok) break;
+      tc_fence_after();
+      tmem_st32(tDPT + grp * 32, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::W_B));
     }
     // ---------------------------------------------------------------- epilogue: dV and scale * dK rows
     const bool store = key < p.Sk;
@@ -416,8 +475,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bar(C::ST_EMPTY + s), 1);
     }
     mbar_init(bar(C::S_FULL), 1);
-    mbar_init(bar(C::P_FULL), 2 * BM);
-    mbar_init(bar(C::RD_DONE), 2 * BM);
+    mbar_init(bar(C::DP_FULL), 1);
+    mbar_init(bar(C::RD_A), 2 * BM);
+    mbar_init(bar(C::RD_B), 2 * BM);
+    mbar_init(bar(C::W_A), 2 * BM);
+    mbar_init(bar(C::W_B), 2 * BM);
     mbar_init(bar(C::ACC_FULL), 1);
     mbar_init(bar(C::DRAIN), 1);
     *abort_flag = 0;
@@ -462,14 +524,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint64_t dStr = sdesc(sStr, 16, 1024);
     const uint64_t dStrMN = sdesc(sStr, BOX_BYTES, 1024);
     constexpr uint32_t TILE16 = C::TILE >> 4;
-    const uint32_t tS = tmem, tDP = tmem + BN, tDQ = tmem + 2 * BN;
-    for (int j = 0; j < nk && ok; ++j) {
-      const uint32_t st = (uint32_t)j % NSTAGE;
-      ok = wait_bar(bar(C::ST_FULL + st), ((uint32_t)j / NSTAGE) & 1u, abort_flag, limit);
-      if (!ok) break;
-      tc_fence_after();
-      const uint64_t k_k = dStr + (uint64_t)(st * 2 * TILE16);
+    // TMEM: S in two buffers (columns [0, 128) and [256 + D, 384 + D)), dP,
+    // dQ.  S(j + 1) and dP(j + 1) are issued as soon as both compute groups
+    // have read S(j) and dP(j), so they run while dS(j) is being written and
+    // dQ += dS(j) K_j follows; S(j + 1) goes to the other buffer, away from
+    // dS(j).
+    const uint32_t tDP = tmem + BN, tDQ = tmem + 2 * BN;
+    auto s_buf = [&](uint32_t j) -> uint32_t { return (j & 1u) ? tmem + 2 * BN + D : tmem; };
+    auto s_dp_products = [&](uint32_t j) {
+      const uint64_t k_k = dStr + (uint64_t)((j % NSTAGE) * 2 * TILE16);
       const uint64_t v_k = k_k + TILE16;
+      const uint32_t tS = s_buf(j);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {   // S = Q K_j^T
         const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
@@ -480,11 +545,29 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
         mma_ss_elect(tDP, dDOd + off, v_k + off, IDESC_S, kk > 0 ? 1u : 0u);
       }
+    };
+    if (ok) ok = wait_bar(bar(C::ST_FULL), 0, abort_flag, limit);
+    if (ok) {
+      tc_fence_after();
+      s_dp_products(0);
       tc_commit_elect(bar(C::S_FULL));
-      ok = wait_bar(bar(C::P_FULL), (uint32_t)j & 1u, abort_flag, limit);
+    }
+    for (uint32_t j = 0; j < (uint32_t)nk && ok; ++j) {
+      const uint32_t st = j % NSTAGE;
+      ok = wait_bar(bar(C::RD_A), j & 1u, abort_flag, limit);     // S(j), dP(j) read
+      if (!ok) break;
+      if (j + 1 < (uint32_t)nk) {
+        ok = wait_bar(bar(C::ST_FULL + (j + 1) % NSTAGE), ((j + 1) / NSTAGE) & 1u, abort_flag, limit);
+        if (!ok) break;
+        tc_fence_after();
+        s_dp_products(j + 1);
+        tc_commit_elect(bar(C::S_FULL));
+      }
+      ok = wait_bar(bar(C::W_A), j & 1u, abort_flag, limit);      // dS(j) written
       if (!ok) break;
       tc_fence_after();
       const uint64_t k_mn = dStrMN + (uint64_t)(st * 2 * TILE16);
+      const uint32_t tS = s_buf(j);
 #pragma unroll
       for (int kk = 0; kk < BN / 16; ++kk)    // dQ += dS K_j
         mma_ts_elect(tDQ, tS + kk * 8, k_mn + (uint64_t)(kk * 128), IDESC_ACC, (j > 0 || kk > 0) ? 1u : 0u);
@@ -500,7 +583,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int rit = quad * 32 + lane;
     const int row = q0 + rit;
     const uint32_t lane_bits = (uint32_t)(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_bits, tDP = tmem + lane_bits + BN, tDQ = tmem + lane_bits + 2 * BN;
+    const uint32_t tDP = tmem + lane_bits + BN, tDQ = tmem + lane_bits + 2 * BN;
     const float c = p.scale_log2;
     const size_t vo = (size_t)bh * p.Sq_pad + (size_t)row;     // padded: in bounds for every row of the tile
     const float lse2 = p.lse2[vo];
@@ -510,6 +593,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = wait_bar(bar(C::S_FULL), (uint32_t)j & 1u, abort_flag, limit);
       if (!ok) break;
       tc_fence_after();
+      const uint32_t tS = tmem + lane_bits + ((j & 1) ? 2 * BN + D : 0);   // this step's S buffer
       const int c0 = j * BN;
       const bool masked = (c0 + BN > p.Sk) || (p.causal && c0 + BN - 1 > q0);
       int lim = p.Sk - 1 - c0;                 // last key (relative) this row sees
@@ -540,14 +624,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       // dS of group g goes over S columns [32 g, 32 g + 32), which group 0
       // reads: both groups finish reading first.
       tc_fence_before();
-      mbar_arrive(bar(C::RD_DONE));
-      ok = wait_bar(bar(C::RD_DONE), (uint32_t)j & 1u, abort_flag, limit);
+      mbar_arrive(bar(C::RD_A));
+      ok = wait_bar(bar(C::RD_A), (uint32_t)j & 1u, abort_flag, limit);
       if (!ok) break;
       tc_fence_after();
       tmem_st32(tS + grp * 32, pd);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(C::P_FULL));
+      mbar_arrive(bar(C::W_A));
     }
     if (ok) ok = wait_bar(bar(C::ACC_FULL), 0, abort_flag, limit);
     if (ok) {
