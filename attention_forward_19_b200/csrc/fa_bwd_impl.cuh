@@ -598,33 +598,32 @@ __global__ void __launch_bounds__(THREADS, 1)
       const bool masked = (c0 + BN > p.Sk) || (p.causal && c0 + BN - 1 > q0);
       int lim = p.Sk - 1 - c0;                 // last key (relative) this row sees
       if (p.causal) lim = min(lim, row - c0);
-      uint32_t pd[32];
-#pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
-        const int col = grp * 64 + ch * 32;    // key columns [col, col + 32)
-        uint32_t s[32], dp[32];
-        tmem_ld32(tS + col, s);
-        tmem_ld32(tDP + col, dp);
-        tmem_wait_ld();
-        reg_fence(s);
-        reg_fence(dp);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int ka = col + 2 * e;
-          float pa = ex2(fmaf(__uint_as_float(s[2 * e]), c, -lse2));
-          float pb = ex2(fmaf(__uint_as_float(s[2 * e + 1]), c, -lse2));
-          if (masked) {
-            if (ka > lim) pa = 0.f;
-            if (ka + 1 > lim) pb = 0.f;
-          }
-          pd[ch * 16 + e] = pack2<BF16>(pa * (__uint_as_float(dp[2 * e]) - dsum),
-                                        pb * (__uint_as_float(dp[2 * e + 1]) - dsum));
-        }
-      }
-      // dS of group g goes over S columns [32 g, 32 g + 32), which group 0
-      // reads: both groups finish reading first.
+      // Read this group's half of S and dP first, then tell the MMA warp:
+      // S(j + 1) and dP(j + 1) run while the exponentials below are computed.
+      uint32_t sv[64], dp[64];
+      tmem_ld32(tS + grp * 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tS + grp * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_ld32(tDP + grp * 64, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+      tmem_ld32(tDP + grp * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+      tmem_wait_ld();
+      reg_fence(sv);
+      reg_fence(dp);
       tc_fence_before();
       mbar_arrive(bar(C::RD_A));
+      uint32_t pd[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int ka = grp * 64 + 2 * e;       // key column within the tile
+        float pa = ex2(fmaf(__uint_as_float(sv[2 * e]), c, -lse2));
+        float pb = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, -lse2));
+        if (masked) {
+          if (ka > lim) pa = 0.f;
+          if (ka + 1 > lim) pb = 0.f;
+        }
+        pd[e] = pack2<BF16>(pa * (__uint_as_float(dp[2 * e]) - dsum), pb * (__uint_as_float(dp[2 * e + 1]) - dsum));
+      }
+      // dS of group g goes over S columns [32 g, 32 g + 32), which group 0
+      // reads: every thread has read (the barrier above), so write now.
       ok = wait_bar(bar(C::RD_A), (uint32_t)j & 1u, abort_flag, limit);
       if (!ok) break;
       tc_fence_after();
