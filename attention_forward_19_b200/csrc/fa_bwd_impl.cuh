@@ -37,6 +37,9 @@ constexpr int THREADS = 320;
 constexpr int LOAD_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr int NSTAGE = 2;      // streamed tile pairs in flight
+// The MMA warp issues step n + 1's first products before step n's last ones
+// (which release step n's stage), so two stages are the minimum.
+static_assert(NSTAGE >= 2, "the overlapped issue order needs two streamed stages");
 
 template <int D>
 struct Cfg {
