@@ -322,11 +322,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       // causal: query q sees this key iff q >= key; only tiles that reach
       // below the key need the test
       const bool masked = p.causal && (q0 < k0 + BM - 1);
-      // ---- phase A: P^T = 2^(s c - lse2) from S^T (kept in fp32 for phase B)
+      // ---- phase A: P^T = 2^(s c - lse2) from S^T, packed to the input dtype
+      // (phase B takes P from these packed words: it is the P the tile
+      // products use, and half the registers of an fp32 copy)
       ok = wait_bar(bar(C::S_FULL), n & 1u, abort_flag, limit);
       if (!ok) break;
       tc_fence_after();
-      float pr[64];
       uint32_t pk[32];
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
@@ -346,8 +347,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (q0 + qa < key) pa = 0.f;
             if (q0 + qa + 1 < key) pb = 0.f;
           }
-          pr[ch * 32 + 2 * e] = pa;
-          pr[ch * 32 + 2 * e + 1] = pb;
           pk[ch * 16 + e] = pack2<BF16>(pa, pb);
         }
       }
@@ -366,6 +365,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = wait_bar(bar(C::DP_FULL), n & 1u, abort_flag, limit);
       if (!ok) break;
       tc_fence_after();
+      uint32_t pg[32];
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
         const int col = grp * 64 + ch * 32;
@@ -378,8 +378,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int qa = col + 2 * e;
           const float4 d4 = *reinterpret_cast<const float4*>(vd + (qa & ~3));
           const float da = (qa & 2) ? d4.z : d4.x, db = (qa & 2) ? d4.w : d4.y;
-          pk[ch * 16 + e] = pack2<BF16>(pr[ch * 32 + 2 * e] * (__uint_as_float(dp[2 * e]) - da),
-                                        pr[ch * 32 + 2 * e + 1] * (__uint_as_float(dp[2 * e + 1]) - db));
+          const float2 pp = unpack2(pk[ch * 16 + e], BF16);
+          pg[ch * 16 + e] = pack2<BF16>(pp.x * (__uint_as_float(dp[2 * e]) - da), pp.y * (__uint_as_float(dp[2 * e + 1]) - db));
         }
       }
       tc_fence_before();
@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = wait_bar(bar(C::RD_B), n & 1u, abort_flag, limit);
       if (!ok) break;
       tc_fence_after();
-      tmem_st32(tDPT + grp * 32, pk);
+      tmem_st32(tDPT + grp * 32, pg);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::W_B));
