@@ -33,11 +33,14 @@ FA_BHSD = 1
 FA_FP16 = 0
 FA_BF16 = 1
 
+FA_MERGE_ACCUMULATE = 1
+FA_MERGE_FINAL = 2
+
 LAYOUTS = {"BSND": FA_BSND, "BHSD": FA_BHSD}
 
 # Names every public symbol of include/fa_fwd.h.
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_noalloc", "fa_fwd_varlen", "fa_bwd",
-                    "fa_bwd_workspace_size",
+                    "fa_bwd_workspace_size", "fa_lse_merge",
                     "fa_selftest_wait_timeout", "fa_device_status", "fa_query_support", "fa_status_string",
                     "fa_last_cuda_error", "fa_version")
 
@@ -87,6 +90,8 @@ def load_library(path=None, rebuild_if_stale=True):
     lib.fa_bwd.restype = c_int
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int,
                            vp, ctypes.c_size_t, vp]
+    lib.fa_lse_merge.restype = c_int
+    lib.fa_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, c_int, c_int, c_int, vp]
     lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_bwd_workspace_size.argtypes = [i64, i64, i64]
     lib.fa_selftest_wait_timeout.restype = c_int
@@ -149,6 +154,13 @@ def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, H, Sq, Sk, D, layout, causal, s
     lib = load_library()
     return lib.fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
                       int(bool(causal)), float(scale), int(dtype), workspace, int(workspace_bytes), stream)
+
+
+def fa_lse_merge(o_part, lse_part, o_acc, lse_acc, o_out, lse_out, B, H, S, D, layout, dtype, flags, stream):
+    """The C fa_lse_merge (merge of a partial attention result) with raw pointers; returns the fa_status code."""
+    lib = load_library()
+    return lib.fa_lse_merge(o_part, lse_part, o_acc, lse_acc, o_out, lse_out, int(B), int(H), int(S), int(D),
+                            int(layout), int(dtype), int(flags), stream)
 
 
 def fa_bwd_workspace_size(B, H, Sq):
@@ -383,6 +395,59 @@ def flash_attention_backward(q, k, v, o, lse, dout, layout="BSND", causal=False,
     if st != FA_OK:
         raise FaError(st, "fa_bwd")
     return dq, dk, dv
+
+
+def lse_merge(o_part, lse_part, o_acc=None, lse_acc=None, out=None, lse_out=None, layout="BSND",
+              accumulate=False, final=False, stream=None):
+    """Merges a partial attention result (o_part, lse_part), normalised over one key block, into the
+    running fp32 result (o_acc, lse_acc) through fa_lse_merge.
+
+    o_part: 16-bit, [B, S, H, D] (BSND) or [B, H, S, D] (BHSD); lse_part fp32 [B, H, S].
+    accumulate=False starts the running result from the partial; accumulate=True merges.  final=True
+    writes the merged result to (out, lse_out) in o_part's dtype (allocated here when None) instead
+    of updating (o_acc, lse_acc).  Returns (o_acc, lse_acc), or (out, lse_out) when final.
+    """
+    import torch
+    lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    if o_part.dim() != 4 or not o_part.is_contiguous():
+        raise ValueError("o_part must be a contiguous 4-D tensor")
+    if lay == FA_BSND:
+        B, S, H, D = o_part.shape
+    else:
+        B, H, S, D = o_part.shape
+    dt = _dtype_code(o_part)
+    if lse_part.shape != (B, H, S) or lse_part.dtype != torch.float32 or not lse_part.is_contiguous():
+        raise ValueError("lse_part must be a contiguous fp32 tensor of shape [B, H, S]")
+    need_acc = accumulate or not final
+    if need_acc:
+        if o_acc is None and not accumulate:
+            o_acc = torch.empty(o_part.shape, dtype=torch.float32, device=o_part.device)
+        if lse_acc is None and not accumulate:
+            lse_acc = torch.empty((B, H, S), dtype=torch.float32, device=o_part.device)
+        if o_acc is None or lse_acc is None:
+            raise ValueError("accumulate=True needs the running result (o_acc, lse_acc)")
+        if o_acc.shape != o_part.shape or o_acc.dtype != torch.float32 or not o_acc.is_contiguous():
+            raise ValueError("o_acc must be a contiguous fp32 tensor shaped like o_part")
+        if lse_acc.shape != (B, H, S) or lse_acc.dtype != torch.float32 or not lse_acc.is_contiguous():
+            raise ValueError("lse_acc must be a contiguous fp32 tensor of shape [B, H, S]")
+    if final:
+        out = torch.empty_like(o_part) if out is None else out
+        lse_out = torch.empty((B, H, S), dtype=torch.float32, device=o_part.device) if lse_out is None else lse_out
+        if out.shape != o_part.shape or out.dtype != o_part.dtype or not out.is_contiguous():
+            raise ValueError("out must be a contiguous tensor like o_part")
+        if lse_out.shape != (B, H, S) or lse_out.dtype != torch.float32 or not lse_out.is_contiguous():
+            raise ValueError("lse_out must be a contiguous fp32 tensor of shape [B, H, S]")
+    if stream is None:
+        stream = torch.cuda.current_stream(o_part.device) if o_part.is_cuda else None
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    flags = (FA_MERGE_ACCUMULATE if accumulate else 0) | (FA_MERGE_FINAL if final else 0)
+    ptr = lambda t: t.data_ptr() if t is not None else None
+    st = fa_lse_merge(o_part.data_ptr(), lse_part.data_ptr(), ptr(o_acc) if need_acc else None,
+                      ptr(lse_acc) if need_acc else None, ptr(out) if final else None,
+                      ptr(lse_out) if final else None, B, H, S, D, lay, dt, flags, sptr)
+    if st != FA_OK:
+        raise FaError(st, "fa_lse_merge")
+    return (out, lse_out) if final else (o_acc, lse_acc)
 
 
 def check_device_status(stream=None):

@@ -248,6 +248,49 @@ fa_status fa_fwd_noalloc(const void *q, const void *k, const void *v, void *o, f
                          fa_layout layout, int causal, float scale, fa_dtype dtype, void *stream);
 
 /*
+ * fa_lse_merge -- merges one partial attention result into a running one.
+ * Attention over a key range split into blocks (ring / context-parallel
+ * attention: page "FlashAttention in ops-transformer on Ascend NPU"
+ * (ai6s.net/6a0d3bfb), section "what else is in the ops-transformer
+ * repository", ring attention for long sequences; page "64K long-sequence
+ * FlashAttention" (ai6s.net/6a140d07), section "performance tuning tips",
+ * multi-card parallelism) gives, per query row, a partial (O_i, LSE_i)
+ * normalised over block i (what fa_fwd writes for that block).  The result over
+ * the union of the blocks follows the online-normalisation update of page
+ * "FlashAttention: long-text inference without running out of memory"
+ * (ai6s.net/6a0d42d8), section on tiling and online normalisation, applied to
+ * whole blocks:
+ *     LSE = log(exp(LSE_acc) + exp(LSE_part))
+ *     O   = exp(LSE_acc - LSE) O_acc + exp(LSE_part - LSE) O_part
+ * A row with LSE = -inf (no visible key in the block) gets weight 0.
+ *
+ * o_part, lse_part  one block's partial: o_part like q (fp16 / bf16, layout
+ *                   `layout`, [B, S, H, D] or [B, H, S, D]), lse_part fp32
+ *                   [B, H, S]; read only
+ * o_acc, lse_acc    the running result in fp32: o_acc with o_part's shape and
+ *                   layout, lse_acc [B, H, S].  Read when flags has
+ *                   FA_MERGE_ACCUMULATE; written (in place) unless flags has
+ *                   FA_MERGE_FINAL.  May be NULL when neither is needed
+ *                   (flags == FA_MERGE_FINAL: a copy of the partial).
+ * o_out, lse_out    written instead of o_acc / lse_acc when flags has
+ *                   FA_MERGE_FINAL: o_out like o_part (rounded to nearest),
+ *                   lse_out fp32 [B, H, S]; else unused (may be NULL)
+ * flags             0: running result = the partial (the first block);
+ *                   FA_MERGE_ACCUMULATE: running result merged with the partial;
+ *                   adding FA_MERGE_FINAL writes the outcome to o_out / lse_out
+ *
+ * The caller owns every buffer.  16-byte alignment for o_part, o_acc, o_out;
+ * 4-byte for the LSE arrays.  D must be 64 or 128.  Outputs must not overlap
+ * any other array (FA_ERR_ALIAS), except that o_acc / lse_acc are updated in
+ * place.  S = 0 is a no-op.  Other errors as for fa_fwd.  Asynchronous on
+ * `stream`.
+ */
+enum { FA_MERGE_ACCUMULATE = 1, FA_MERGE_FINAL = 2 };
+fa_status fa_lse_merge(const void *o_part, const float *lse_part, float *o_acc, float *lse_acc,
+                       void *o_out, float *lse_out, int64_t B, int64_t H, int64_t S, int64_t D,
+                       fa_layout layout, fa_dtype dtype, int flags, void *stream);
+
+/*
  * fa_device_status -- synchronises `stream`, then reads and clears the
  * library's device-side error word on the current device.  Returns FA_OK,
  * FA_ERR_TIMEOUT if a kernel stopped at a wait limit since the last call,

@@ -239,3 +239,39 @@ def test_bwd_host_validation(lib):
     assert call_bwd(dq=Q) == fa.FA_ERR_ALIAS
     assert call_bwd(dk=DV) == fa.FA_ERR_ALIAS
     assert call_bwd(ws=DO_) == fa.FA_ERR_ALIAS
+
+
+# fa_lse_merge: fake pointers far apart, sized for B=1, H=2, S=64, D=128
+MP, MLP, MA, MLA, MO, MLO = (1 << 40, 2 << 40, 3 << 40, 4 << 40, 5 << 40, 6 << 40)
+
+
+def call_merge(o_part=MP, lse_part=MLP, o_acc=MA, lse_acc=MLA, o_out=MO, lse_out=MLO, B=1, H=2, S=64, D=128,
+               layout=fa.FA_BSND, dtype=fa.FA_BF16, flags=fa.FA_MERGE_ACCUMULATE | fa.FA_MERGE_FINAL):
+    return fa.fa_lse_merge(o_part, lse_part, o_acc, lse_acc, o_out, lse_out, B, H, S, D, layout, dtype, flags,
+                           None)
+
+
+def test_merge_host_validation(lib):
+    for kw in (dict(B=0), dict(H=-1), dict(S=-1), dict(layout=3), dict(dtype=7), dict(flags=4), dict(flags=-1),
+               dict(o_part=0), dict(lse_part=0), dict(o_acc=0), dict(lse_acc=0), dict(o_out=0),
+               dict(lse_out=0), dict(o_acc=0, flags=fa.FA_MERGE_ACCUMULATE), dict(o_acc=0, flags=0),
+               dict(o_out=0, flags=fa.FA_MERGE_FINAL)):
+        assert call_merge(**kw) == fa.FA_ERR_INVALID_ARG, kw
+    assert call_merge(D=96) == fa.FA_ERR_UNSUPPORTED
+    assert call_merge(S=0) == fa.FA_OK
+    assert call_merge(o_part=MP + 8) == fa.FA_ERR_MISALIGNED
+    assert call_merge(o_acc=MA + 4) == fa.FA_ERR_MISALIGNED
+    assert call_merge(o_out=MO + 2) == fa.FA_ERR_MISALIGNED
+    assert call_merge(lse_acc=MLA + 2) == fa.FA_ERR_MISALIGNED
+    assert call_merge(o_out=MP) == fa.FA_ERR_ALIAS
+    assert call_merge(lse_out=MA + 64) == fa.FA_ERR_ALIAS
+    assert call_merge(o_acc=MP + 4096) == fa.FA_ERR_ALIAS
+    assert call_merge(lse_acc=MA + 16) == fa.FA_ERR_ALIAS
+
+
+def test_merge_optional_buffers_are_not_checked(lib):
+    # a final copy (flags = FINAL) needs no running result; a first merge (flags = 0) needs no output:
+    # with everything else valid the call reaches the device checks, which fail on fake pointers
+    for kw in (dict(o_acc=0, lse_acc=0, flags=fa.FA_MERGE_FINAL), dict(o_out=0, lse_out=0, flags=0)):
+        st = call_merge(**kw)
+        assert st not in (fa.FA_ERR_INVALID_ARG, fa.FA_ERR_MISALIGNED, fa.FA_ERR_ALIAS), (kw, st)

@@ -1,0 +1,195 @@
+"""Host logic of ring (context-parallel) attention, on the CPU.
+
+The schedule, the sharding and the exchange of attention_forward_19_b200.ring
+run here with the two compute steps supplied by the oracle (attention of one
+block, and the merge of partial results), in fp64, so that any wrong block,
+mask, source rank or merge order shows as a large error.  The ranks are either
+emulated in one process or run as gloo processes exchanging chunks through
+torch.distributed.
+"""
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from attention_forward_19_b200 import ring
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+class OracleOps:
+    """Block attention and merge from the oracle, in fp64 on the CPU."""
+
+    acc_dtype = torch.float64
+    lse_dtype = torch.float64
+
+    def __init__(self, layout, scale):
+        from oracle import attn as oracle_attn
+        self.layout, self.scale, self.orc = layout, scale, oracle_attn.default()
+        self.calls = []
+
+    def _to_layout(self, o_bhsd):
+        t = torch.from_numpy(o_bhsd)
+        return t.permute(0, 2, 1, 3) if self.layout == "BSND" else t
+
+    def _head_major(self, t):
+        return (t.permute(0, 2, 1, 3) if self.layout == "BSND" else t).double().numpy()
+
+    def block(self, q, k, v, diagonal, o, lse):
+        self.calls.append(bool(diagonal))
+        oo, ll = self.orc.fwd(q, k, v, layout=self.layout, causal=bool(diagonal), scale=self.scale)
+        o.copy_(self._to_layout(oo))
+        lse.copy_(torch.from_numpy(ll))
+
+    def merge(self, o_part, lse_part, o_acc, lse_acc, o_out, lse_out, accumulate, final):
+        from oracle.merge import merge_partials
+        parts = [self._head_major(o_part)]
+        lses = [lse_part.double().numpy()]
+        if accumulate:
+            parts.insert(0, self._head_major(o_acc))
+            lses.insert(0, lse_acc.double().numpy())
+        o, l = merge_partials(parts, lses)
+        dst_o, dst_l = (o_out, lse_out) if final else (o_acc, lse_acc)
+        dst_o.copy_(self._to_layout(o))
+        dst_l.copy_(torch.from_numpy(l))
+
+
+def _qkv(layout, B=1, H=2, S=48, D=16, seed=5):
+    g = torch.Generator().manual_seed(seed)
+    shape = (B, S, H, D) if layout == "BSND" else (B, H, S, D)
+    return [torch.randn(shape, generator=g, dtype=torch.float64) for _ in range(3)]
+
+
+def _oracle_whole(q, k, v, layout, causal, scale):
+    from oracle import attn as oracle_attn
+    o, l = oracle_attn.default().fwd(q, k, v, layout=layout, causal=causal, scale=scale)
+    o = torch.from_numpy(o)
+    return (o.permute(0, 2, 1, 3) if layout == "BSND" else o), torch.from_numpy(l)
+
+
+# ----------------------------------------------------------------------------- schedule
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+def test_zigzag_chunks_partition_the_sequence(world):
+    ids = [c for r in range(world) for c in ring.zigzag_chunk_ids(r, world)]
+    assert sorted(ids) == list(range(2 * world))
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_every_visible_key_is_used_exactly_once(world, causal):
+    # expand the chunk-level plan to element level and compare with the mask itself
+    Sc = 3
+    S = 2 * world * Sc
+    count = np.zeros((S, S), dtype=int)
+    for r in range(world):
+        plan = ring.contribution_plan(r, world, causal)
+        mine = ring.zigzag_chunk_ids(r, world)
+        for i, blocks in enumerate(plan):
+            assert blocks[0][3] and blocks[-1][4]
+            assert sum(b[3] for b in blocks) == 1 and sum(b[4] for b in blocks) == 1
+            for (t, j, diag, _, _) in blocks:
+                c = ring.zigzag_chunk_ids(ring.ring_source(r, world, t), world)[j]
+                a = mine[i]
+                for qi in range(Sc):
+                    for kj in range(Sc):
+                        if diag and kj > qi:
+                            continue
+                        count[a * Sc + qi, c * Sc + kj] += 1
+    mask = np.tril(np.ones((S, S), dtype=int)) if causal else np.ones((S, S), dtype=int)
+    assert np.array_equal(count, mask)
+
+
+def test_zigzag_balances_causal_work():
+    world = 4
+    work = []
+    for r in range(world):
+        plan = ring.contribution_plan(r, world, True)
+        work.append(sum(0.5 if d else 1.0 for blocks in plan for (_, _, d, _, _) in blocks))
+    assert len(set(work)) == 1
+
+
+@pytest.mark.parametrize("layout", ["BSND", "BHSD"])
+def test_shard_unshard_round_trip(layout):
+    x = _qkv(layout, S=24)[0]
+    parts = [ring.shard(x, r, 3, layout) for r in range(3)]
+    assert all(p.is_contiguous() and p.shape[0] == 2 for p in parts)
+    assert torch.equal(ring.unshard(parts, layout), x)
+    with pytest.raises(ValueError):
+        ring.shard(x, 0, 5, layout)            # 24 rows are not a multiple of 10
+
+
+# ----------------------------------------------------------------------------- emulated ranks, oracle compute
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("layout", ["BSND", "BHSD"])
+def test_emulated_ring_with_oracle_steps_matches_whole_attention(world, causal, layout):
+    q, k, v = _qkv(layout, S=2 * world * 6)
+    scale = 0.3
+    ops = OracleOps(layout, scale)
+    o, l = ring.ring_attention_emulated(q, k, v, world, causal=causal, scale=scale, layout=layout, ops=ops)
+    o_ref, l_ref = _oracle_whole(q, k, v, layout, causal, scale)
+    assert float((o - o_ref).abs().max()) < 1e-12
+    assert float((l - l_ref).abs().max()) < 1e-12
+    n_blocks = (2 * world) * (2 * world + 1) // 2 if causal else (2 * world) ** 2
+    assert len(ops.calls) == n_blocks
+    assert sum(ops.calls) == (2 * world if causal else 0)   # one diagonal block per chunk
+
+
+# ----------------------------------------------------------------------------- gloo ranks
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _gloo_worker(rank, world, port, layout, causal, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        from attention_forward_19_b200 import ring as ring_mod
+        q, k, v = _qkv(layout, S=2 * world * 5)
+        mine = [ring_mod.shard(t, rank, world, layout) for t in (q, k, v)]
+        ops = OracleOps(layout, 0.25)
+        o, l = ring_mod.ring_steps(*mine, rank, world, ring_mod.P2PExchange(), ops, causal)
+        out[rank] = (o.numpy(), l.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,causal,layout", [(2, True, "BSND"), (3, True, "BHSD"), (2, False, "BHSD")])
+def test_gloo_ring_exchange_matches_whole_attention(world, causal, layout):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    procs = [ctx.Process(target=_gloo_worker, args=(r, world, port, layout, causal, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = dict(out)
+    o = ring.unshard([torch.from_numpy(res[r][0]) for r in range(world)], layout)
+    l = ring.unshard([torch.from_numpy(res[r][1]) for r in range(world)], layout, seq_dim=2)
+    q, k, v = _qkv(layout, S=2 * world * 5)
+    o_ref, l_ref = _oracle_whole(q, k, v, layout, causal, 0.25)
+    assert float((o - o_ref).abs().max()) < 1e-12
+    assert float((l - l_ref).abs().max()) < 1e-12
