@@ -40,7 +40,7 @@ LAYOUTS = {"BSND": FA_BSND, "BHSD": FA_BHSD}
 
 # Names every public symbol of include/fa_fwd.h.
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_noalloc", "fa_fwd_varlen", "fa_bwd",
-                    "fa_bwd_workspace_size", "fa_lse_merge",
+                    "fa_bwd_workspace_size", "fa_lse_merge", "fa_out_proj", "fa_fwd_proj",
                     "fa_selftest_wait_timeout", "fa_device_status", "fa_query_support", "fa_status_string",
                     "fa_last_cuda_error", "fa_version")
 
@@ -92,6 +92,11 @@ def load_library(path=None, rebuild_if_stale=True):
                            vp, ctypes.c_size_t, vp]
     lib.fa_lse_merge.restype = c_int
     lib.fa_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, c_int, c_int, c_int, vp]
+    lib.fa_out_proj.restype = c_int
+    lib.fa_out_proj.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, vp]
+    lib.fa_fwd_proj.restype = c_int
+    lib.fa_fwd_proj.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, c_int, c_int, c_float,
+                                c_int, vp, ctypes.c_size_t, vp]
     lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_bwd_workspace_size.argtypes = [i64, i64, i64]
     lib.fa_selftest_wait_timeout.restype = c_int
@@ -161,6 +166,20 @@ def fa_lse_merge(o_part, lse_part, o_acc, lse_acc, o_out, lse_out, B, H, S, D, l
     lib = load_library()
     return lib.fa_lse_merge(o_part, lse_part, o_acc, lse_acc, o_out, lse_out, int(B), int(H), int(S), int(D),
                             int(layout), int(dtype), int(flags), stream)
+
+
+def fa_out_proj(o, w_o, y, B, H, S, D, E, layout, dtype, stream):
+    """The C fa_out_proj (y = o w_o^T) with raw pointers and sizes; returns the fa_status code."""
+    return load_library().fa_out_proj(o, w_o, y, int(B), int(H), int(S), int(D), int(E), int(layout), int(dtype),
+                                      stream)
+
+
+def fa_fwd_proj(q, k, v, w_o, o, lse, y, B, H, Sq, Sk, D, E, layout, causal, scale, dtype, workspace,
+                workspace_bytes, stream):
+    """The C fa_fwd_proj (attention, then y = o w_o^T) with raw pointers; returns the fa_status code."""
+    return load_library().fa_fwd_proj(q, k, v, w_o, o, lse, y, int(B), int(H), int(Sq), int(Sk), int(D), int(E),
+                                      int(layout), int(bool(causal)), float(scale), int(dtype), workspace,
+                                      int(workspace_bytes), stream)
 
 
 def fa_bwd_workspace_size(B, H, Sq):
@@ -448,6 +467,77 @@ def lse_merge(o_part, lse_part, o_acc=None, lse_acc=None, out=None, lse_out=None
     if st != FA_OK:
         raise FaError(st, "fa_lse_merge")
     return (out, lse_out) if final else (o_acc, lse_acc)
+
+
+def _proj_dims(o, w_o, lay):
+    if o.dim() != 4 or not o.is_contiguous():
+        raise ValueError("o must be a contiguous 4-D tensor")
+    if lay == FA_BSND:
+        B, S, H, D = o.shape
+    else:
+        B, H, S, D = o.shape
+    if w_o.dim() != 2 or w_o.shape[1] != H * D or not w_o.is_contiguous() or w_o.dtype != o.dtype:
+        raise ValueError(f"w_o must be a contiguous [E, H * D = {H * D}] tensor of o's dtype")
+    return B, H, S, D, w_o.shape[0]
+
+
+def out_projection(o, w_o, layout="BSND", y=None, stream=None):
+    """y = o w_o^T through fa_out_proj: o [B, S, H, D] (BSND) or [B, H, S, D] (BHSD), w_o [E, H * D]
+    (a linear layer's weight).  Returns y [B, S, E] in o's dtype."""
+    import torch
+    lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    B, H, S, D, E = _proj_dims(o, w_o, lay)
+    if y is None:
+        y = torch.empty((B, S, E), dtype=o.dtype, device=o.device)
+    if y.shape != (B, S, E) or y.dtype != o.dtype or not y.is_contiguous():
+        raise ValueError(f"y must be a contiguous [{B}, {S}, {E}] tensor of o's dtype")
+    if stream is None:
+        stream = torch.cuda.current_stream(o.device) if o.is_cuda else None
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    st = fa_out_proj(o.data_ptr(), w_o.data_ptr(), y.data_ptr(), B, H, S, D, E, lay, _dtype_code(o), sptr)
+    if st != FA_OK:
+        raise FaError(st, "fa_out_proj")
+    return y
+
+
+def flash_attention_forward_proj(q, k, v, w_o, layout="BSND", causal=False, scale=None, out=None, lse=None, y=None,
+                                 stream=None, workspace=None):
+    """Attention followed by its output projection (fa_fwd_proj): returns (y, o, lse) with
+    y = o w_o^T [B, Sq, E], o and lse as flash_attention_forward returns them."""
+    import torch
+    lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    B, H, Sq, Sk, D = _dims(q, k, lay)
+    if v.shape != k.shape:
+        raise ValueError(f"v {tuple(v.shape)} must have k's shape {tuple(k.shape)}")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_contiguous() or t.dtype != q.dtype:
+            raise ValueError(f"{name} must be contiguous and share q's dtype")
+    if w_o.dim() != 2 or w_o.shape[1] != H * D or not w_o.is_contiguous() or w_o.dtype != q.dtype:
+        raise ValueError(f"w_o must be a contiguous [E, H * D = {H * D}] tensor of q's dtype")
+    E = w_o.shape[0]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device) if lse is None else lse
+    y = torch.empty((B, Sq, E), dtype=q.dtype, device=q.device) if y is None else y
+    if out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor like q")
+    if lse.shape != (B, H, Sq) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 tensor of shape [B, H, Sq]")
+    if y.shape != (B, Sq, E) or y.dtype != q.dtype or not y.is_contiguous():
+        raise ValueError(f"y must be a contiguous [{B}, {Sq}, {E}] tensor of q's dtype")
+    nbytes = fa_fwd_workspace_size()
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device) if q.is_cuda else None
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    st = fa_fwd_proj(q.data_ptr(), k.data_ptr(), v.data_ptr(), w_o.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                     y.data_ptr(), B, H, Sq, Sk, D, E, lay, causal, scale, _dtype_code(q), workspace.data_ptr(),
+                     workspace.numel() * workspace.element_size(), sptr)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_proj")
+    return y, out, lse
 
 
 def check_device_status(stream=None):

@@ -1549,3 +1549,4 @@ int fa_version(void) { return FA_VERSION; }
 // The backward pass (gradients) shares this translation unit's helpers.
 #include "fa_bwd_impl.cuh"
 #include "fa_merge_impl.cuh"
+#include "fa_proj_impl.cuh"

@@ -19,6 +19,14 @@ on a bounded row sample of the same workload, each step one sample.
 and lse) on the same workload instead, and prints its own JSON line; its
 metric counts 2.5x the forward's flops (five tile products to the forward's
 two, the usual convention), kernel time only.
+
+--ring times ring (context-parallel) attention instead: ONE sequence split
+over the N ranks (strong scaling; default workload bf16 BHSD B=1 H=8
+S=65536 D=128 causal), each rank holding its zigzag pair of chunks and
+passing key/value chunks on over NCCL point-to-point.  A step is the whole
+ring; the time is the max over ranks and the value the whole sequence's
+flops / that time.  With N = 1 the ring has one rank (its two chunks, three
+blocks and one merge).
 """
 import argparse
 import hashlib
@@ -165,9 +173,15 @@ def oracle_sample(w, target_s, max_rows=None, threads=0):
 # ----------------------------------------------------------------------------- native arm
 
 
+RING_WORKLOAD = "bf16_bhsd_b1_h8_s65536_d128_causal"
+
+
 def bench_workload(args):
     """The timed workload; --workload / --bh select another one (profiling runs only)."""
-    w = WORKLOADS[args.workload]
+    name = args.workload
+    if name is None:
+        name = RING_WORKLOAD if getattr(args, "ring", False) else BENCH_WORKLOAD
+    w = WORKLOADS[name]
     if args.bh:
         b, h = (int(x) for x in args.bh.split(","))
         w = w.with_(B=b, H=h, name=f"{w.name}_b{b}_h{h}")
@@ -382,6 +396,72 @@ def run_backward(args, rank, world, local_rank):
     }
 
 
+def run_ring(args, rank, world, local_rank):
+    """Times ring attention of one sequence over the ranks (strong scaling; one JSON line)."""
+    import attention_forward_19_b200 as fa
+    from attention_forward_19_b200 import ring
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = bench_workload(args)
+    if w.Sq != w.Sk or w.Sq % (2 * world):
+        raise SystemExit(f"--ring needs Sq == Sk and a multiple of {2 * world} rows")
+    q, k, v = make_qkv(w)                       # the same whole sequence on every rank, then its shard
+    q, k, v = (ring.shard(t, rank, world, w.layout).to(dev) for t in (q, k, v))
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return ring.ring_attention_forward(q, k, v, causal=w.causal, scale=w.scale, layout=w.layout)
+
+    for _ in range(args.warmup):
+        step()
+    fa.check_device_status(stream)
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(cvd.split(",")[local_rank].strip() if cvd else str(local_rank))
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    fa.check_device_status(stream)
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ms_step = ms_total / args.steps
+    flops = w.flops()
+    value = flops * args.steps / (ms_total * 1e-3) / 1e12
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    plan = ring.contribution_plan(0, world, w.causal)
+    blocks = sum(len(p) for p in plan)
+    merges = sum(len(p) for p in plan if len(p) > 1)
+    cfg = workload_config(w, world)
+    cfg.update({"global_batch": w.B, "parallelism": f"cp{world} (ring over NCCL point-to-point, zigzag chunks)"})
+    return {
+        "metric": "ring attn fwd TFLOP/s (causal-halved, one sequence over all ranks)", "value": value,
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": cfg,
+        "roofline": {"bound": "tensor", "achieved": value / world, "peak": peak, "unit": UNIT,
+                     "frac": value / world / peak, "traffic": None,
+                     "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
+                                    if peak_kind == "measured" else "fallback 1590 TFLOP/s",
+                     "note": "per-GPU share of the whole sequence's flops over the slowest rank's time"},
+        "gpu_launches": (blocks + merges) * args.steps,
+        "gpu_launches_note": f"rank 0 per step: {blocks} fa_fwd block launches and {merges} fa_lse_merge launches",
+        "clocks": clk,
+    }
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 
@@ -423,9 +503,11 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="time the kernel only (profiling runs)")
-    ap.add_argument("--workload", choices=list(WORKLOADS), default=BENCH_WORKLOAD)
+    ap.add_argument("--workload", choices=list(WORKLOADS), default=None,
+                    help=f"default {BENCH_WORKLOAD} ({RING_WORKLOAD} with --ring)")
     ap.add_argument("--bh", default=None, help="override B,H of the workload (profiling runs)")
     ap.add_argument("--backward", action="store_true", help="time the backward pass instead (its own JSON line)")
+    ap.add_argument("--ring", action="store_true", help="time ring attention of one sequence over the ranks")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -442,7 +524,8 @@ def main():
             torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                                  device_id=torch.device("cuda", local_rank))
         try:
-            line = (run_backward if args.backward else run_native)(args, rank, world, local_rank)
+            run = run_ring if args.ring else run_backward if args.backward else run_native
+            line = run(args, rank, world, local_rank)
         finally:
             if world > 1:
                 torch.distributed.destroy_process_group()

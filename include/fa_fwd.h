@@ -291,6 +291,41 @@ fa_status fa_lse_merge(const void *o_part, const float *lse_part, float *o_acc, 
                        fa_layout layout, fa_dtype dtype, int flags, void *stream);
 
 /*
+ * fa_out_proj -- the attention output projection Y = O W^T (page "catlass
+ * FlashAttention template tuning" (hwcomputing.csdn.net/6a0d4681), section on
+ * graph fusion: the fused operator FusedAttnProj is FlashAttention followed by
+ * the output MatMul).  Every token's heads form one row of inputs:
+ *     y[b, s, n] = sum_{h, d} o[b, s, h, d] * w_o[n, h * D + d]
+ * fp32 accumulation on the tensor cores, y rounded to nearest in dtype.
+ *
+ * o      attention output as fa_fwd writes it: [B, S, H, D] (FA_BSND) or
+ *        [B, H, S, D] (FA_BHSD), fp16 / bf16, 16-byte aligned; read only
+ * w_o    [E, H * D] row-major (a linear layer's weight: row n is output
+ *        feature n), same dtype, 16-byte aligned; read only
+ * y      [B, S, E] row-major, same dtype, 16-byte aligned, fully overwritten
+ * E      output features, a positive multiple of 32
+ *
+ * Caller-owned buffers; y must not overlap o or w_o (FA_ERR_ALIAS).  S = 0 is
+ * a no-op.  D must be 64 or 128 and E a multiple of 32 (else
+ * FA_ERR_UNSUPPORTED).  Other errors as for fa_fwd.  Asynchronous on `stream`.
+ */
+fa_status fa_out_proj(const void *o, const void *w_o, void *y, int64_t B, int64_t H, int64_t S, int64_t D,
+                      int64_t E, fa_layout layout, fa_dtype dtype, void *stream);
+
+/*
+ * fa_fwd_proj -- attention followed by its output projection in one call:
+ * fa_fwd_ws (or fa_fwd when workspace is NULL) writes o and lse, then
+ * fa_out_proj writes y = o w_o^T, stream-ordered on `stream`.  Arguments as
+ * for those two calls (Sq for S); o is caller-owned and also an output (the
+ * attention result, kept for a backward pass).  y and w_o must not overlap
+ * any other array.
+ */
+fa_status fa_fwd_proj(const void *q, const void *k, const void *v, const void *w_o, void *o, float *lse, void *y,
+                      int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D, int64_t E, fa_layout layout,
+                      int causal, float scale, fa_dtype dtype, void *workspace, size_t workspace_bytes,
+                      void *stream);
+
+/*
  * fa_device_status -- synchronises `stream`, then reads and clears the
  * library's device-side error word on the current device.  Returns FA_OK,
  * FA_ERR_TIMEOUT if a kernel stopped at a wait limit since the last call,

@@ -275,3 +275,36 @@ def test_merge_optional_buffers_are_not_checked(lib):
     for kw in (dict(o_acc=0, lse_acc=0, flags=fa.FA_MERGE_FINAL), dict(o_out=0, lse_out=0, flags=0)):
         st = call_merge(**kw)
         assert st not in (fa.FA_ERR_INVALID_ARG, fa.FA_ERR_MISALIGNED, fa.FA_ERR_ALIAS), (kw, st)
+
+
+def call_out_proj(o=MP, w=MA, y=MO, B=1, H=2, S=64, D=128, E=256, layout=fa.FA_BSND, dtype=fa.FA_BF16):
+    return fa.fa_out_proj(o, w, y, B, H, S, D, E, layout, dtype, None)
+
+
+def test_out_proj_host_validation(lib):
+    for kw in (dict(B=0), dict(H=0), dict(S=-1), dict(E=0), dict(layout=2), dict(dtype=5), dict(o=0), dict(w=0),
+               dict(y=0)):
+        assert call_out_proj(**kw) == fa.FA_ERR_INVALID_ARG, kw
+    assert call_out_proj(D=32) == fa.FA_ERR_UNSUPPORTED
+    assert call_out_proj(E=48) == fa.FA_ERR_UNSUPPORTED          # not a multiple of 32
+    assert call_out_proj(S=0) == fa.FA_OK
+    assert call_out_proj(o=MP + 8) == fa.FA_ERR_MISALIGNED
+    assert call_out_proj(y=MO + 2) == fa.FA_ERR_MISALIGNED
+    assert call_out_proj(y=MP + 64) == fa.FA_ERR_ALIAS
+    assert call_out_proj(w=MO + 1024) == fa.FA_ERR_ALIAS
+
+
+def test_fwd_proj_host_validation(lib):
+    def call(**kw):
+        a = dict(q=Q, k=K, v=V, w=MA, o=O, lse=L, y=MO, B=1, H=2, Sq=64, Sk=64, D=128, E=256, layout=fa.FA_BSND,
+                 causal=0, scale=0.125, dtype=fa.FA_BF16)
+        a.update(kw)
+        return fa.fa_fwd_proj(a["q"], a["k"], a["v"], a["w"], a["o"], a["lse"], a["y"], a["B"], a["H"], a["Sq"],
+                              a["Sk"], a["D"], a["E"], a["layout"], a["causal"], a["scale"], a["dtype"], None, 0,
+                              None)
+    assert call(w=0) == fa.FA_ERR_INVALID_ARG
+    assert call(y=0) == fa.FA_ERR_INVALID_ARG
+    assert call(E=40) == fa.FA_ERR_UNSUPPORTED
+    assert call(y=Q) == fa.FA_ERR_ALIAS
+    assert call(w=O) == fa.FA_ERR_ALIAS
+    assert call(scale=float("inf")) == fa.FA_ERR_INVALID_ARG
