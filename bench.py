@@ -27,6 +27,11 @@ passing key/value chunks on over NCCL point-to-point.  A step is the whole
 ring; the time is the max over ranks and the value the whole sequence's
 flops / that time.  With N = 1 the ring has one rank (its two chunks, three
 blocks and one merge).
+
+--proj times attention followed by its output projection (fa_fwd_proj:
+y = o w_o^T with E = H * D output features, w_o seeded N(0, 1/(H D))) on the
+same workload; the value counts both parts' flops, and the attention kernel
+and the projection kernel are also timed alone (events around each).
 """
 import argparse
 import hashlib
@@ -73,7 +78,8 @@ def workload_config(w, n_gpus):
         "workload": w.name, "model": "attention forward (no weights)", "B": w.B, "H": w.H, "Sq": w.Sq,
         "Sk": w.Sk, "D": w.D, "layout": w.layout, "causal": w.causal, "scale": w.scale, "dtype": w.dtype,
         "global_batch": w.B * n_gpus, "seq_len": w.Sq, "parallelism": f"dp{n_gpus} (independent heads per rank)",
-        "l2": "no flush: inputs 3 x 168 MB > 126 MB L2",
+        "l2": (f"no flush: inputs 3 x {w.B * w.H * w.Sq * w.D * 2 / 1e6:.0f} MB > 126 MB L2"
+               if w.B * w.H * w.Sq * w.D * 2 > 126e6 else "no flush: the inputs fit in L2 (a latency-bound case)"),
         "inputs": "seeded N(0,1), fp32 randn rounded to bf16",
     }
 
@@ -462,6 +468,92 @@ def run_ring(args, rank, world, local_rank):
     }
 
 
+def run_proj(args, rank, world, local_rank):
+    """Times attention + output projection (fa_fwd_proj) and each kernel alone (one JSON line)."""
+    import attention_forward_19_b200 as fa
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w0 = bench_workload(args)
+    w = rank_workload(w0, rank)
+    q, k, v = make_qkv(w, device=dev)
+    E = w.H * w.D
+    g = torch.Generator(device="cpu").manual_seed(w.seed + 600)
+    w_o = (torch.randn((E, w.H * w.D), generator=g) / math.sqrt(w.H * w.D)).to(q.dtype).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
+    y = torch.empty((w.B, w.Sq, E), dtype=q.dtype, device=dev)
+    ws = torch.empty(fa.fa_fwd_workspace_size(), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fused():
+        fa.flash_attention_forward_proj(q, k, v, w_o, layout=w.layout, causal=w.causal, scale=w.scale, out=o,
+                                        lse=lse, y=y, stream=stream, workspace=ws)
+
+    def attn():
+        fa.flash_attention_forward(q, k, v, layout=w.layout, causal=w.causal, scale=w.scale, out=o, lse=lse,
+                                   stream=stream, workspace=ws)
+
+    def proj():
+        fa.out_projection(o, w_o, layout=w.layout, y=y, stream=stream)
+
+    def timed(fn, steps):
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        return max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+
+    for _ in range(args.warmup):
+        fused()
+    fa.check_device_status(stream)
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(cvd.split(",")[local_rank].strip() if cvd else str(local_rank))
+    clocks.start()
+    time.sleep(0.3)
+    ms_step = timed(fused, args.steps)
+    clk = clocks.stop()
+    ms_attn = timed(attn, max(3, args.steps // 2))
+    ms_proj = timed(proj, max(3, args.steps // 2))
+    fa.check_device_status(stream)
+    f_attn = w.flops()
+    f_proj = 2.0 * w.B * w.Sq * w.H * w.D * E
+    value = world * (f_attn + f_proj) / (ms_step * 1e-3) / 1e12
+    if rank != 0:
+        return None
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    src = (f"{peak_kind} bf16 burst (MEASURED_PEAKS.json bf16_tflops)" if peak_kind == "measured"
+           else "fallback 1590 TFLOP/s")
+    a_attn = f_attn / (ms_attn * 1e-3) / 1e12
+    a_proj = f_proj / (ms_proj * 1e-3) / 1e12
+    cfg = workload_config(w0, world)
+    cfg.update({"model": "attention forward + output projection (random-init w_o, E = H * D)", "E": E})
+    return {
+        "metric": "attn fwd + out-proj TFLOP/s (causal-halved attention flops + 2 B S (H D) E)", "value": value,
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": cfg,
+        "roofline": {"bound": "tensor", "achieved": a_attn, "peak": peak, "unit": UNIT, "frac": a_attn / peak,
+                     "traffic": None, "peak_source": src, "kernel": "fa_fwd_kernel (dominant), timed alone",
+                     "ms_per_launch": ms_attn},
+        "roofline_proj": {"bound": "tensor", "achieved": a_proj, "peak": peak, "unit": UNIT,
+                          "frac": a_proj / peak, "traffic": None, "peak_source": src,
+                          "kernel": "proj_kernel (fa_out_proj), timed alone", "ms_per_launch": ms_proj,
+                          "algorithmic_flops_per_launch": f_proj},
+        "gpu_launches": 2 * args.steps,
+        "gpu_launches_note": "per step: one fa_fwd_kernel and one proj_kernel launch",
+        "clocks": clk,
+    }
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 
@@ -508,6 +600,7 @@ def main():
     ap.add_argument("--bh", default=None, help="override B,H of the workload (profiling runs)")
     ap.add_argument("--backward", action="store_true", help="time the backward pass instead (its own JSON line)")
     ap.add_argument("--ring", action="store_true", help="time ring attention of one sequence over the ranks")
+    ap.add_argument("--proj", action="store_true", help="time attention + output projection (fa_fwd_proj)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -524,7 +617,8 @@ def main():
             torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                                  device_id=torch.device("cuda", local_rank))
         try:
-            run = run_ring if args.ring else run_backward if args.backward else run_native
+            run = (run_ring if args.ring else run_proj if args.proj else run_backward if args.backward
+                   else run_native)
             line = run(args, rank, world, local_rank)
         finally:
             if world > 1:
