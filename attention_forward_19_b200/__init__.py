@@ -40,7 +40,8 @@ LAYOUTS = {"BSND": FA_BSND, "BHSD": FA_BHSD}
 
 # Names every public symbol of include/fa_fwd.h.
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_noalloc", "fa_fwd_varlen", "fa_bwd",
-                    "fa_bwd_workspace_size", "fa_lse_merge", "fa_out_proj", "fa_fwd_proj",
+                    "fa_bwd_workspace_size", "fa_bwd_atomic",
+                    "fa_bwd_atomic_workspace_size", "fa_lse_merge", "fa_out_proj", "fa_fwd_proj",
                     "fa_selftest_wait_timeout", "fa_device_status", "fa_query_support", "fa_status_string",
                     "fa_last_cuda_error", "fa_version")
 
@@ -97,6 +98,10 @@ def load_library(path=None, rebuild_if_stale=True):
     lib.fa_fwd_proj.restype = c_int
     lib.fa_fwd_proj.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, c_int, c_int, c_float,
                                 c_int, vp, ctypes.c_size_t, vp]
+    lib.fa_bwd_atomic.restype = c_int
+    lib.fa_bwd_atomic.argtypes = lib.fa_bwd.argtypes
+    lib.fa_bwd_atomic_workspace_size.restype = ctypes.c_size_t
+    lib.fa_bwd_atomic_workspace_size.argtypes = [i64, i64, i64, i64]
     lib.fa_bwd_workspace_size.restype = ctypes.c_size_t
     lib.fa_bwd_workspace_size.argtypes = [i64, i64, i64]
     lib.fa_selftest_wait_timeout.restype = c_int
@@ -180,6 +185,19 @@ def fa_fwd_proj(q, k, v, w_o, o, lse, y, B, H, Sq, Sk, D, E, layout, causal, sca
     return load_library().fa_fwd_proj(q, k, v, w_o, o, lse, y, int(B), int(H), int(Sq), int(Sk), int(D), int(E),
                                       int(layout), int(bool(causal)), float(scale), int(dtype), workspace,
                                       int(workspace_bytes), stream)
+
+
+def fa_bwd_atomic(q, k, v, o, dout, lse, dq, dk, dv, B, H, Sq, Sk, D, layout, causal, scale, dtype, workspace,
+                  workspace_bytes, stream):
+    """The C fa_bwd_atomic (non-deterministic dQ accumulation) with raw pointers; returns the fa_status code."""
+    lib = load_library()
+    return lib.fa_bwd_atomic(q, k, v, o, dout, lse, dq, dk, dv, int(B), int(H), int(Sq), int(Sk), int(D),
+                             int(layout), int(bool(causal)), float(scale), int(dtype), workspace,
+                             int(workspace_bytes), stream)
+
+
+def fa_bwd_atomic_workspace_size(B, H, Sq, D):
+    return load_library().fa_bwd_atomic_workspace_size(int(B), int(H), int(Sq), int(D))
 
 
 def fa_bwd_workspace_size(B, H, Sq):
@@ -373,13 +391,16 @@ def flash_attention_varlen_forward(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seql
 
 
 def flash_attention_backward(q, k, v, o, lse, dout, layout="BSND", causal=False, scale=None, dq=None, dk=None,
-                             dv=None, stream=None, workspace=None):
+                             dv=None, stream=None, workspace=None, deterministic=True):
     """Gradients (dq, dk, dv) of flash_attention_forward through the C ABI.
 
     q, k, v as for the forward; o and lse as the forward returned them; dout
     (dL/dO) like o.  Returns (dq, dk, dv) shaped like q, k, v.  `workspace`, a
-    uint8 CUDA tensor of fa_bwd_workspace_size(B, H, Sq) bytes, is allocated
-    here when not given.  Runs on `stream` without synchronising.
+    uint8 CUDA tensor of fa_bwd_workspace_size(B, H, Sq) bytes
+    (fa_bwd_atomic_workspace_size(B, H, Sq, D) when deterministic=False), is
+    allocated here when not given.  deterministic=False calls fa_bwd_atomic
+    (D = 128): one kernel per key tile, dQ added up in fp32 in any order.
+    Runs on `stream` without synchronising.
     """
     import torch
     lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
@@ -401,18 +422,19 @@ def flash_attention_backward(q, k, v, o, lse, dout, layout="BSND", causal=False,
     for name, t, like in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
         if t.shape != like.shape or t.dtype != like.dtype or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous tensor like {name[1:]}")
-    nbytes = fa_bwd_workspace_size(B, H, Sq)
+    nbytes = fa_bwd_workspace_size(B, H, Sq) if deterministic else fa_bwd_atomic_workspace_size(B, H, Sq, D)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
     wbytes = workspace.numel() * workspace.element_size()
     if stream is None:
         stream = torch.cuda.current_stream(q.device) if q.is_cuda else None
     sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
-    st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
-                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, Sq, Sk, D, lay, causal, scale, dt,
-                workspace.data_ptr(), wbytes, sptr)
+    fn = fa_bwd if deterministic else fa_bwd_atomic
+    st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, Sq, Sk, D, lay, causal, scale, dt,
+            workspace.data_ptr(), wbytes, sptr)
     if st != FA_OK:
-        raise FaError(st, "fa_bwd")
+        raise FaError(st, "fa_bwd" if deterministic else "fa_bwd_atomic")
     return dq, dk, dv
 
 

@@ -1,0 +1,504 @@
+// fa_bwd_atomic_impl.cuh -- the non-deterministic backward pass: dK, dV and dQ
+// from one kernel per key tile, dQ added up across key tiles in fp32.
+// Included at the end of fa_fwd.cu after fa_bwd_impl.cuh (whose prep kernel,
+// parameters and helpers it uses).
+//
+// Page "catlass FlashAttention template tuning" (hwcomputing.csdn.net/6a0d4681),
+// section on the backward: the `deterministic` switch chooses between an
+// ordered accumulation and atomic adds, the latter being faster; results then
+// differ from run to run by the order of the additions.  The arithmetic is the
+// same as fa_bwd's (P = 2^(S c - LSE2), dS = P (dP - D), dV = P^T dO,
+// dK = scale dS^T Q, dQ = scale dS K).
+//
+// One CTA per 128-key tile walks the visible queries in steps of 64 (D = 128):
+//   S^T = K Q_u^T, dP^T = V dO_u^T         (keys on the TMEM lanes, 64 columns each)
+//   dV += P^T dO_u, dK += dS^T Q_u         (A from TMEM, as in fa_bwd)
+//   dQ_u^T = K^T dS_u^T                    (both operands from shared memory:
+//                                           K^T is the K tile read MN-major, dS^T
+//                                           is written there by the compute warps)
+// TMEM: dV [0,128) | dK [128,256) | S^T [256,320) | dP^T [320,384) |
+// dQ^T [384,448) and [448,512) (two buffers).  The compute warps read each
+// dQ_u^T tile (lanes = head-dim index), stage it in shared memory as 64 rows x
+// 128 fp32 and add it to the fp32 accumulator in global memory with one bulk
+// reduction (cp.reduce.async.bulk .add.f32, 32 KB).  A last kernel scales the
+// accumulator and rounds it into dq.  The 64-query step keeps the TMEM budget
+// at 512 columns; the stream of Q / dO sub-tiles has three stages.
+
+namespace fa {
+namespace bwda {
+
+using bwd::LOAD_WARP;
+using bwd::MMA_WARP;
+using bwd::THREADS;
+
+constexpr int DH = 128;          // head dim of this kernel
+constexpr int SUB = 64;          // queries per step
+constexpr int NST = 3;           // streamed stages (a Q and a dO sub-tile, two vectors)
+constexpr int SUB_BOX = SUB * 128;            // one 64-row x 64-element box: 8 KB
+constexpr int TILE = BM * DH * 2;             // the K or V tile: 32 KB
+constexpr int SUBT = SUB * DH * 2;            // a Q or dO sub-tile: 16 KB
+constexpr int IN_FULL = 0;
+constexpr int ST_FULL = 1;
+constexpr int ST_EMPTY = ST_FULL + NST;
+constexpr int S_FULL = ST_EMPTY + NST;
+constexpr int DP_FULL = S_FULL + 1;
+constexpr int DQ_FULL = DP_FULL + 1;          // two: dQ^T buffer 0 / 1 complete
+constexpr int RD_A = DQ_FULL + 2;             // both groups have read S^T (256 arrivals)
+constexpr int RD_B = RD_A + 1;                // ... dP^T (256)
+constexpr int W_A = RD_B + 1;                 // P^T written (256)
+constexpr int W_B = W_A + 1;                  // dS^T written to TMEM and shared memory (256)
+constexpr int RD_C = W_B + 1;                 // two: a dQ^T buffer read (256)
+constexpr int STG_FREE = RD_C + 2;            // the staging tile may be written (1)
+constexpr int STG_FULL = STG_FREE + 1;        // the staging tile is written (256)
+constexpr int ACC_FULL = STG_FULL + 1;
+constexpr int DRAIN = ACC_FULL + 1;
+constexpr int NBAR = DRAIN + 1;
+constexpr int SMEM_FIX = 0;                               // K tile, V tile
+constexpr int SMEM_STREAM = 2 * TILE;                     // per stage: Q_u, dO_u sub-tiles
+constexpr int SMEM_DST = SMEM_STREAM + NST * 2 * SUBT;    // dS^T: 128 keys x 64 queries, 16-bit, swizzled
+constexpr int SMEM_STG = SMEM_DST + BM * SUB * 2;         // dQ^T staging: 64 queries x 128 fp32
+constexpr int SMEM_VEC = SMEM_STG + SUB * DH * 4;         // per stage: lse2[64], dsum[64]
+constexpr int SMEM_BAR = SMEM_VEC + NST * 2 * SUB * 4;
+constexpr int SMEM_MISC = SMEM_BAR + NBAR * 8;
+constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;
+static_assert(SMEM_DST % 1024 == 0, "the swizzled dS^T tile needs 1024-byte alignment");
+static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
+
+constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_ST = 256, COL_DPT = 320, COL_DQ = 384;
+
+// Instruction descriptor (kind::f16) with both operands' majorness given.
+__host__ __device__ constexpr uint32_t idesc_ab(int M, int N, uint32_t fmt, uint32_t a_mn, uint32_t b_mn) {
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | (a_mn << 15) | (b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_reduce_add_f32(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// The two 64-row boxes of one Q / dO sub-tile (rows s0 .. s0 + 63 of head h, batch b).
+__device__ __forceinline__ void load_sub(uint32_t dst, const CUtensorMap* map, uint32_t bar, int bhsd, int s0, int h,
+                                         int b) {
+#pragma unroll
+  for (int bx = 0; bx < DH / 64; ++bx)
+    tma_load_4d(dst + bx * SUB_BOX, map, bar, bx * 64, bhsd ? s0 : h, bhsd ? h : s0, b);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(THREADS, 1)
+    dkdvq_kernel(const __grid_constant__ bwd::Params p, const __grid_constant__ CUtensorMap tmQ64,
+                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmDO64) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sFix = smem_u32(smem + SMEM_FIX);
+  const uint32_t sStr = smem_u32(smem + SMEM_STREAM);
+  const uint32_t sDst = smem_u32(smem + SMEM_DST);
+  const uint32_t sStg = smem_u32(smem + SMEM_STG);
+  const float* sVec = reinterpret_cast<const float*>(smem + SMEM_VEC);
+  const uint32_t bars = smem_u32(smem + SMEM_BAR);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SMEM_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SMEM_MISC + 4);
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t limit = p.wait_limit_ns;
+
+  // longest first: the first key tiles see the most queries (causal)
+  const int bhs = p.B * p.H;
+  const int kt = blockIdx.x / bhs;
+  const int bh = blockIdx.x - kt * bhs;
+  const int b = bh / p.H, h = bh - b * p.H;
+  const int k0 = kt * BN;
+  const int t64 = (p.Sq + SUB - 1) / SUB;
+  const int u_begin = p.causal ? k0 / SUB : 0;      // the first 64-query sub-tile with a row >= k0
+  const int nu = max(0, t64 - u_begin);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(IN_FULL), 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(bar(ST_FULL + s), 1);
+      mbar_init(bar(ST_EMPTY + s), 1);
+    }
+    mbar_init(bar(S_FULL), 1);
+    mbar_init(bar(DP_FULL), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(DQ_FULL + i), 1);
+      mbar_init(bar(RD_C + i), 2 * BM);
+    }
+    mbar_init(bar(RD_A), 2 * BM);
+    mbar_init(bar(RD_B), 2 * BM);
+    mbar_init(bar(W_A), 2 * BM);
+    mbar_init(bar(W_B), 2 * BM);
+    mbar_init(bar(STG_FREE), 1);
+    mbar_init(bar(STG_FULL), 2 * BM);
+    mbar_init(bar(ACC_FULL), 1);
+    mbar_init(bar(DRAIN), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  constexpr uint32_t FMT = BF16 ? 1u : 0u;
+  constexpr uint32_t IDESC_ST = idesc_ab(BM, SUB, FMT, 0, 0);    // 128 keys x 64 queries, both K-major
+  constexpr uint32_t IDESC_ACC = idesc_ab(BM, DH, FMT, 0, 1);    // 128 keys x D, A in TMEM, B MN-major
+  constexpr uint32_t IDESC_DQ = idesc_ab(DH, SUB, FMT, 1, 1);    // D x 64 queries, A and B MN-major
+
+  if (warp == LOAD_WARP) {
+    if (lane == 0 && nu > 0) {
+      bool ok = true;
+      mbar_arrive_expect_tx(bar(IN_FULL), 2 * TILE);
+      bwd::load_tile(sFix, &tmK, bar(IN_FULL), DH / 64, p.bhsd, k0, h, b);
+      bwd::load_tile(sFix + TILE, &tmV, bar(IN_FULL), DH / 64, p.bhsd, k0, h, b);
+      uint32_t issued = 0;
+      for (int u = 0; u < nu && ok; ++u, ++issued) {
+        const uint32_t st = issued % NST;
+        ok = wait_bar1(bar(ST_EMPTY + st), ((issued / NST) & 1u) ^ 1u, abort_flag, limit);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(ST_FULL + st), 2 * SUBT + 2 * SUB * 4);
+        const uint32_t dst = sStr + st * 2 * SUBT;
+        const int q0 = (u_begin + u) * SUB;
+        load_sub(dst, &tmQ64, bar(ST_FULL + st), p.bhsd, q0, h, b);
+        load_sub(dst + SUBT, &tmDO64, bar(ST_FULL + st), p.bhsd, q0, h, b);
+        const size_t vo = (size_t)bh * p.Sq_pad + (size_t)q0;
+        const uint32_t vdst = smem_u32(sVec + st * 2 * SUB);
+        bwd::bulk_load(vdst, p.lse2 + vo, SUB * 4, bar(ST_FULL + st));
+        bwd::bulk_load(vdst + SUB * 4, p.dsum + vo, SUB * 4, bar(ST_FULL + st));
+      }
+      drain_wait(bar(IN_FULL), 0, limit);
+      const uint32_t first = issued > (uint32_t)NST ? issued - NST : 0u;
+      for (uint32_t c = first; c < issued; ++c) drain_wait(bar(ST_FULL + c % NST), (c / NST) & 1u, limit);
+    }
+    __syncwarp();
+  } else if (warp == MMA_WARP) {
+    if (nu > 0) {
+      bool ok = wait_bar(bar(IN_FULL), 0, abort_flag, limit);
+      const uint64_t dKk = sdesc(sFix, 16, 1024), dVk = sdesc(sFix + TILE, 16, 1024);
+      const uint64_t dKmn = sdesc(sFix, BOX_BYTES, 1024);         // K^T: the K tile read MN-major
+      const uint64_t dStrK = sdesc(sStr, 16, 1024);               // a sub-tile, K-major
+      const uint64_t dStrMN = sdesc(sStr, SUB_BOX, 1024);         // a sub-tile, MN-major
+      const uint64_t dDst = sdesc(sDst, SUB_BOX, 1024);           // dS^T, MN-major (one 64-query group)
+      constexpr uint32_t SUBT16 = SUBT >> 4;
+      const uint32_t tST = tmem + COL_ST, tDPT = tmem + COL_DPT, tDV = tmem + COL_DV, tDK = tmem + COL_DK;
+      auto kmajor_products = [&](uint32_t d_tmem, uint64_t a, uint64_t bsub) {   // 128 x 64 over K = D
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t offa = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
+          const uint32_t offb = (uint32_t)((kk >> 2) * (SUB_BOX >> 4) + (kk & 3) * 2);
+          mma_ss_elect(d_tmem, a + offa, bsub + offb, IDESC_ST, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto q_k = [&](uint32_t u) { return dStrK + (uint64_t)((u % NST) * 2 * SUBT16); };
+      auto do_k = [&](uint32_t u) { return dStrK + (uint64_t)((u % NST) * 2 * SUBT16 + SUBT16); };
+      // Order of the tensor work: S^T(0), dP^T(0), then per step u
+      //   dV(u), S^T(u+1), dK(u), dP^T(u+1), dQ^T(u)
+      // S^T(u+1) overwrites P^T(u) and dP^T(u+1) overwrites dS^T(u) only after
+      // the products that read them (tcgen05 MMAs run in issue order).
+      if (ok) ok = wait_bar(bar(ST_FULL), 0, abort_flag, limit);
+      if (ok) {
+        tc_fence_after();
+        kmajor_products(tST, dKk, q_k(0));
+        tc_commit_elect(bar(S_FULL));
+        kmajor_products(tDPT, dVk, do_k(0));
+        tc_commit_elect(bar(DP_FULL));
+      }
+      for (uint32_t u = 0; u < (uint32_t)nu && ok; ++u) {
+        const uint32_t st = u % NST;
+        const uint64_t q_mn = dStrMN + (uint64_t)(st * 2 * SUBT16);
+        const uint64_t do_mn = q_mn + SUBT16;
+        ok = wait_bar(bar(W_A), u & 1u, abort_flag, limit);        // P^T(u) written
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < SUB / 16; ++kk)   // dV += P^T dO_u
+          mma_ts_elect(tDV, tST + kk * 8, do_mn + (uint64_t)(kk * 128), IDESC_ACC, (u > 0 || kk > 0) ? 1u : 0u);
+        const bool more = u + 1 < (uint32_t)nu;
+        if (more) {
+          ok = wait_bar(bar(ST_FULL + (u + 1) % NST), ((u + 1) / NST) & 1u, abort_flag, limit);
+          if (!ok) break;
+          tc_fence_after();
+          kmajor_products(tST, dKk, q_k(u + 1));
+          tc_commit_elect(bar(S_FULL));
+        }
+        ok = wait_bar(bar(W_B), u & 1u, abort_flag, limit);        // dS^T(u) written
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < SUB / 16; ++kk)   // dK += dS^T Q_u
+          mma_ts_elect(tDK, tDPT + kk * 8, q_mn + (uint64_t)(kk * 128), IDESC_ACC, (u > 0 || kk > 0) ? 1u : 0u);
+        tc_commit_elect(bar(ST_EMPTY + st));
+        if (more) {
+          kmajor_products(tDPT, dVk, do_k(u + 1));
+          tc_commit_elect(bar(DP_FULL));
+        }
+        const uint32_t qb = u & 1u;
+        if (u >= 2) {                            // the compute warps have read dQ^T(u - 2) from this buffer
+          ok = wait_bar(bar(RD_C + qb), ((u >> 1) - 1) & 1u, abort_flag, limit);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        const uint32_t tDQ = tmem + COL_DQ + qb * SUB;
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)    // dQ^T = K^T dS^T(u)
+          mma_ss_elect(tDQ, dKmn + (uint64_t)(kk * 128), dDst + (uint64_t)(kk * 128), IDESC_DQ, kk > 0 ? 1u : 0u);
+        tc_commit_elect(bar(DQ_FULL + qb));
+      }
+      if (ok) tc_commit_elect(bar(ACC_FULL));
+      tc_commit_elect(bar(DRAIN));
+      if (lane == 0) drain_wait(bar(DRAIN), 0, limit);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- compute: one thread per key (phases A, B),
+    // one per head-dim index (phase C); group g takes queries [32 g, 32 g + 32) of a step
+    const int quad = warp & 3, grp = warp >> 2;
+    const int rit = quad * 32 + lane;
+    const int key = k0 + rit;
+    const bool key_live = key < p.Sk;
+    const uint32_t lane_bits = (uint32_t)(quad * 32) << 16;
+    const uint32_t tST = tmem + lane_bits + COL_ST, tDPT = tmem + lane_bits + COL_DPT;
+    const uint32_t tDV = tmem + lane_bits + COL_DV, tDK = tmem + lane_bits + COL_DK;
+    const float c = p.scale_log2;
+    const bool leader = threadIdx.x == 0;
+    float* dq_acc_bh = p.dq_acc + (size_t)bh * p.Sq_pad * DH;
+    bool ok = true;
+    // phase C of step v: dQ^T(v) -> staging -> one bulk reduction into the accumulator
+    auto phase_c = [&](uint32_t v) -> bool {
+      if (leader) {
+        bulk_wait_read0();                     // the previous reduction has read the staging tile
+        mbar_arrive(bar(STG_FREE));
+      }
+      if (!wait_bar(bar(STG_FREE), v & 1u, abort_flag, limit)) return false;
+      if (!wait_bar(bar(DQ_FULL + (v & 1u)), (v >> 1) & 1u, abort_flag, limit)) return false;
+      tc_fence_after();
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_bits + COL_DQ + (v & 1u) * SUB + grp * 32, r);
+      tmem_wait_ld();
+      reg_fence(r);
+      tc_fence_before();
+      mbar_arrive(bar(RD_C + (v & 1u)));
+      // staging [64 queries][128] fp32: this thread's head-dim index is rit
+      float* stg = reinterpret_cast<float*>(smem + SMEM_STG);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) stg[(grp * 32 + j) * DH + rit] = __uint_as_float(r[j]);
+      fence_proxy_async_smem();
+      mbar_arrive(bar(STG_FULL));
+      bool lok = true;
+      if (leader) {
+        lok = wait_bar1(bar(STG_FULL), v & 1u, abort_flag, limit);
+        if (lok) {
+          const int q0 = (u_begin + (int)v) * SUB;
+          bulk_reduce_add_f32(dq_acc_bh + (size_t)q0 * DH, sStg, SUB * DH * 4);
+          bulk_commit();
+        }
+      }
+      if (warp == 0) lok = __shfl_sync(0xffffffffu, lok, 0);   // keep the warp's result uniform
+      return lok;
+    };
+    for (uint32_t u = 0; u < (uint32_t)nu && ok; ++u) {
+      const uint32_t st = u % NST;
+      ok = wait_bar(bar(ST_FULL + st), (u / NST) & 1u, abort_flag, limit);   // the vectors came by bulk copy
+      if (!ok) break;
+      const float* vl = sVec + st * 2 * SUB;
+      const float* vd = vl + SUB;
+      const int q0 = (u_begin + (int)u) * SUB;
+      const bool masked = p.causal && (q0 < k0 + BM - 1);
+      // ---- phase A: P^T = 2^(s c - lse2), packed
+      ok = wait_bar(bar(S_FULL), u & 1u, abort_flag, limit);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t pk[16];
+      {
+        uint32_t sv[32];
+        tmem_ld32(tST + grp * 32, sv);
+        tmem_wait_ld();
+        reg_fence(sv);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int qa = grp * 32 + 2 * e;
+          const float2 l2 = *reinterpret_cast<const float2*>(vl + qa);
+          float pa = ex2(fmaf(__uint_as_float(sv[2 * e]), c, -l2.x));
+          float pb = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, -l2.y));
+          if (masked) {
+            if (q0 + qa < key) pa = 0.f;
+            if (q0 + qa + 1 < key) pb = 0.f;
+          }
+          if (!key_live) pa = pb = 0.f;         // keys past Sk (zero-filled rows) take no weight
+          pk[e] = pack2<BF16>(pa, pb);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(RD_A));
+      ok = wait_bar(bar(RD_A), u & 1u, abort_flag, limit);
+      if (!ok) break;
+      tc_fence_after();
+      tmem_st16(tST + grp * 16, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(W_A));
+      // ---- phase B: dS^T = P^T (dP^T - D), to TMEM (for dK) and to shared memory (for dQ)
+      ok = wait_bar(bar(DP_FULL), u & 1u, abort_flag, limit);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t pg[16];
+      {
+        uint32_t dp[32];
+        tmem_ld32(tDPT + grp * 32, dp);
+        tmem_wait_ld();
+        reg_fence(dp);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int qa = grp * 32 + 2 * e;
+          const float2 d2 = *reinterpret_cast<const float2*>(vd + qa);
+          const float2 pp = bwd::unpack2(pk[e], BF16);
+          pg[e] = pack2<BF16>(pp.x * (__uint_as_float(dp[2 * e]) - d2.x), pp.y * (__uint_as_float(dp[2 * e + 1]) - d2.y));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(RD_B));
+      ok = wait_bar(bar(RD_B), u & 1u, abort_flag, limit);
+      if (!ok) break;
+      tc_fence_after();
+      tmem_st16(tDPT + grp * 16, pg);
+      if (u >= 1) {                            // dQ^T(u - 1) has finished reading the shared dS^T tile
+        ok = wait_bar(bar(DQ_FULL + ((u - 1) & 1u)), ((u - 1) >> 1) & 1u, abort_flag, limit);
+        if (!ok) break;
+      }
+      {
+        // row rit of the 128 x 64 tile, 16-byte chunks 4 grp .. 4 grp + 3, 128-byte swizzle
+        uint8_t* row = smem + SMEM_DST + rit * 128;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int chunk = (grp * 4 + j) ^ (rit & 7);
+          *reinterpret_cast<uint4*>(row + chunk * 16) = make_uint4(pg[4 * j], pg[4 * j + 1], pg[4 * j + 2], pg[4 * j + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(W_B));
+      // ---- phase C of the previous step
+      if (u >= 1) {
+        ok = phase_c(u - 1);
+        if (!ok) break;
+      }
+    }
+    if (ok && nu > 0) ok = phase_c((uint32_t)nu - 1);
+    if (leader) bulk_wait0();                  // every reduction issued has completed
+    // ---------------------------------------------------------------- epilogue: dV and scale * dK rows
+    const bool store = key < p.Sk;
+    uint8_t* dvrow = p.dv + (size_t)b * p.k_bs + (size_t)h * p.k_hs + (size_t)key * p.k_rs;
+    uint8_t* dkrow = p.dk + (size_t)b * p.k_bs + (size_t)h * p.k_hs + (size_t)key * p.k_rs;
+    uint8_t* dst = grp ? dkrow : dvrow;
+    if (nu == 0) {
+      if (store) {
+#pragma unroll
+        for (int e = 0; e < DH * 2 / 16; ++e) reinterpret_cast<uint4*>(dst)[e] = make_uint4(0, 0, 0, 0);
+      }
+    } else if (ok) {
+      ok = wait_bar(bar(ACC_FULL), 0, abort_flag, limit);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t src = grp ? tDK : tDV;
+        const float f = grp ? p.scale : 1.f;
+#pragma unroll
+        for (int q4 = 0; q4 < DH / 32; ++q4) {
+          uint32_t r[32];
+          tmem_ld32(src + q4 * 32, r);
+          tmem_wait_ld();
+          reg_fence(r);
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) w[e] = pack2<BF16>(__uint_as_float(r[2 * e]) * f, __uint_as_float(r[2 * e + 1]) * f);
+          if (store) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              reinterpret_cast<uint4*>(dst + q4 * 64)[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// dq = scale * accumulator, rounded to the input dtype: one warp per query row, four columns per lane.
+template <bool BF16>
+__global__ void __launch_bounds__(256) dq_convert_kernel(const __grid_constant__ bwd::Params p) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const long long total = (long long)p.B * p.H * p.Sq;
+  if (row >= total) return;
+  const int bh = (int)(row / p.Sq);
+  const int i = (int)(row - (long long)bh * p.Sq);
+  const int b = bh / p.H, h = bh - b * p.H;
+  const float4 a = *reinterpret_cast<const float4*>(p.dq_acc + ((size_t)bh * p.Sq_pad + i) * DH + lane * 4);
+  uint8_t* dst = p.dq + (size_t)b * p.q_bs + (size_t)h * p.q_hs + (size_t)i * p.q_rs + lane * 8;
+  *reinterpret_cast<uint2*>(dst) = make_uint2(pack2<BF16>(a.x * p.scale, a.y * p.scale),
+                                              pack2<BF16>(a.z * p.scale, a.w * p.scale));
+}
+
+}  // namespace bwda
+}  // namespace fa
+
+// ============================================================================= host side (atomic backward)
+
+namespace {
+
+bool g_bwda_configured[kMaxDevices][2];
+
+template <bool BF16>
+fa_status launch_bwd_atomic(fa::bwd::Params& prm, const CUtensorMap& mq64, const CUtensorMap& mk,
+                            const CUtensorMap& mv, const CUtensorMap& mdo64, int dev, cudaStream_t s) {
+  auto kern = fa::bwda::dkdvq_kernel<BF16>;
+  {
+    std::lock_guard<std::mutex> g(g_dev_mu);
+    if (!g_bwda_configured[dev][BF16 ? 1 : 0]) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::bwda::SMEM_BYTES);
+      if (e != cudaSuccess) return cuda_fail((int)e);
+      g_bwda_configured[dev][BF16 ? 1 : 0] = true;
+    }
+  }
+  const long long rows = (long long)prm.B * prm.H * prm.Sq_pad;
+  fa::bwd::prep_kernel<128, BF16><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail((int)e);
+  e = cudaMemsetAsync(prm.dq_acc, 0, (size_t)rows * 128 * sizeof(float), s);
+  if (e != cudaSuccess) return cuda_fail((int)e);
+  kern<<<(unsigned)(prm.B * prm.H * prm.tk), fa::bwd::THREADS, fa::bwda::SMEM_BYTES, s>>>(prm, mq64, mk, mv, mdo64);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail((int)e);
+  const long long qrows = (long long)prm.B * prm.H * prm.Sq;
+  fa::bwda::dq_convert_kernel<BF16><<<(unsigned)((qrows + 7) / 8), 256, 0, s>>>(prm);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail((int)e);
+  return FA_OK;
+}
+
+}  // namespace

@@ -82,6 +82,7 @@ struct Params {
   int causal, bhsd;
   float scale, scale_log2;
   unsigned long long wait_limit_ns;
+  float* dq_acc;            // non-deterministic variant: fp32 dQ accumulator [B * H, Sq_pad, D]
 };
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -671,6 +672,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 }  // namespace bwd
 }  // namespace fa
 
+// The non-deterministic variant (dQ added across key tiles) shares the prep
+// kernel, the parameters and the host checks.
+#include "fa_bwd_atomic_impl.cuh"
+
 // ============================================================================= host side (backward)
 
 namespace {
@@ -720,10 +725,17 @@ size_t fa_bwd_workspace_size(int64_t B, int64_t H, int64_t Sq) {
   return (size_t)(2 * B * H * bwd_sq_pad(Sq)) * sizeof(float);
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-                 void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D,
-                 fa_layout layout, int causal, float scale, fa_dtype dtype, void* workspace,
-                 size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+size_t bwd_atomic_workspace_size(int64_t B, int64_t H, int64_t Sq, int64_t D);
+
+// Validation, tensor maps and parameters shared by fa_bwd and fa_bwd_atomic.
+fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D,
+                   fa_layout layout, int causal, float scale, fa_dtype dtype, void* workspace,
+                   size_t workspace_bytes, void* stream, bool atomic) {
   // ---- arguments that need no device
   if (B <= 0 || H <= 0 || Sq < 0 || Sk <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
   if (layout != FA_BSND && layout != FA_BHSD) return FA_ERR_INVALID_ARG;
@@ -757,7 +769,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
       15u)
     return FA_ERR_MISALIGNED;
   if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA_ERR_MISALIGNED;
-  const size_t wbytes = fa_bwd_workspace_size(B, H, Sq);
+  if (atomic && D != 128) return FA_ERR_UNSUPPORTED;
+  const size_t wbytes = atomic ? bwd_atomic_workspace_size(B, H, Sq, D) : fa_bwd_workspace_size(B, H, Sq);
   if (workspace_bytes < wbytes) return FA_ERR_INVALID_ARG;
   const void* outs[4] = {dq, dk, dv, workspace};
   const size_t out_bytes[4] = {qbytes, kvbytes, kvbytes, wbytes};
@@ -817,12 +830,50 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   prm.scale = scale;
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   prm.wait_limit_ns = 1000000000ull;
+  prm.dq_acc = nullptr;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (atomic) {
+    prm.dq_acc = static_cast<float*>(workspace) + 2 * B * H * sq_pad;
+    CUtensorMap mq64, mdo64;
+    if ((st = make_map(&mq64, q, dtype, layout, B, H, Sq, D, fa::bwda::SUB)) != FA_OK) return st;
+    if ((st = make_map(&mdo64, dout, dtype, layout, B, H, Sq, D, fa::bwda::SUB)) != FA_OK) return st;
+    return dtype == FA_BF16 ? launch_bwd_atomic<true>(prm, mq64, mk, mv, mdo64, dev, s)
+                            : launch_bwd_atomic<false>(prm, mq64, mk, mv, mdo64, dev, s);
+  }
   if (D == 128)
     return dtype == FA_BF16 ? launch_bwd<128, true>(prm, mq, mk, mv, mdo, dev, s, 0)
                             : launch_bwd<128, false>(prm, mq, mk, mv, mdo, dev, s, 1);
   return dtype == FA_BF16 ? launch_bwd<64, true>(prm, mq, mk, mv, mdo, dev, s, 2)
                           : launch_bwd<64, false>(prm, mq, mk, mv, mdo, dev, s, 3);
+}
+
+size_t bwd_atomic_workspace_size(int64_t B, int64_t H, int64_t Sq, int64_t D) {
+  if (B <= 0 || H <= 0 || Sq <= 0 || D <= 0) return 0;
+  return (size_t)(B * H * bwd_sq_pad(Sq)) * (size_t)(2 + D) * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                 void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D,
+                 fa_layout layout, int causal, float scale, fa_dtype dtype, void* workspace,
+                 size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, Sq, Sk, D, layout, causal, scale, dtype, workspace,
+                  workspace_bytes, stream, false);
+}
+
+size_t fa_bwd_atomic_workspace_size(int64_t B, int64_t H, int64_t Sq, int64_t D) {
+  return bwd_atomic_workspace_size(B, H, Sq, D);
+}
+
+fa_status fa_bwd_atomic(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                        const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Sq,
+                        int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(q, k, v, o, dout, lse, dq, dk, dv, B, H, Sq, Sk, D, layout, causal, scale, dtype, workspace,
+                  workspace_bytes, stream, true);
 }
 
 }  // extern "C"

@@ -1108,9 +1108,9 @@ EncodeTiledFn get_encode_fn(int* err) {
 }
 
 // A [B, S, H, D] (BSND) or [B, H, S, D] (BHSD) tensor seen as 4-D for TMA,
-// dims in memory order, 128-row x 64-column boxes with a 128-byte swizzle.
+// dims in memory order, box_rows x 64-column boxes with a 128-byte swizzle.
 fa_status make_map(CUtensorMap* map, const void* base, fa_dtype dt, fa_layout lay, int64_t B, int64_t H,
-                   int64_t S, int64_t D) {
+                   int64_t S, int64_t D, int box_rows = fa::BM) {
   int err = 0;
   EncodeTiledFn enc = get_encode_fn(&err);
   if (!enc) return cuda_fail(err);
@@ -1120,11 +1120,11 @@ fa_status make_map(CUtensorMap* map, const void* base, fa_dtype dt, fa_layout la
   if (lay == FA_BHSD) {
     dims[0] = D; dims[1] = S; dims[2] = H; dims[3] = B;
     strides[0] = D * 2; strides[1] = S * D * 2; strides[2] = H * S * D * 2;
-    box[0] = 64; box[1] = fa::BM; box[2] = 1; box[3] = 1;
+    box[0] = 64; box[1] = (cuuint32_t)box_rows; box[2] = 1; box[3] = 1;
   } else {
     dims[0] = D; dims[1] = H; dims[2] = S; dims[3] = B;
     strides[0] = D * 2; strides[1] = H * D * 2; strides[2] = S * H * D * 2;
-    box[0] = 64; box[1] = 1; box[2] = fa::BM; box[3] = 1;
+    box[0] = 64; box[1] = 1; box[2] = (cuuint32_t)box_rows; box[3] = 1;
   }
   const CUtensorMapDataType t =
       dt == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;

@@ -18,7 +18,8 @@ on a bounded row sample of the same workload, each step one sample.
 --backward times the backward pass (fa_bwd: dq, dk, dv from the forward's o
 and lse) on the same workload instead, and prints its own JSON line; its
 metric counts 2.5x the forward's flops (five tile products to the forward's
-two, the usual convention), kernel time only.
+two, the usual convention), kernel time only.  --backward --atomic times
+the non-deterministic variant (fa_bwd_atomic: dQ added up across key tiles).
 
 --ring times ring (context-parallel) attention instead: ONE sequence split
 over the N ranks (strong scaling; default workload bf16 BHSD B=1 H=8
@@ -349,11 +350,13 @@ def run_backward(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     o, lse = fa.flash_attention_forward(q, k, v, layout=w.layout, causal=w.causal, scale=w.scale, stream=stream)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(max(16, fa.fa_bwd_workspace_size(w.B, w.H, w.Sq)), dtype=torch.uint8, device=dev)
+    det = not args.atomic
+    nbytes = fa.fa_bwd_workspace_size(w.B, w.H, w.Sq) if det else fa.fa_bwd_atomic_workspace_size(w.B, w.H, w.Sq, w.D)
+    ws = torch.empty(max(16, nbytes), dtype=torch.uint8, device=dev)
 
     def step():
         fa.flash_attention_backward(q, k, v, o, lse, do, layout=w.layout, causal=w.causal, scale=w.scale, dq=dq,
-                                    dk=dk, dv=dv, stream=stream, workspace=ws)
+                                    dk=dk, dv=dv, stream=stream, workspace=ws, deterministic=det)
 
     for _ in range(args.warmup):
         step()
@@ -386,7 +389,8 @@ def run_backward(args, rank, world, local_rank):
     peak = float(peaks["bf16_tflops"])
     achieved = flops / (ms_step * 1e-3) / 1e12
     return {
-        "metric": "attn bwd TFLOP/s (2.5x the causal-halved forward flops)", "value": value, "unit": UNIT,
+        "metric": "attn bwd TFLOP/s (2.5x the causal-halved forward flops)"
+                  + ("" if det else ", non-deterministic variant"), "value": value, "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": workload_config(w0, world),
@@ -395,9 +399,11 @@ def run_backward(args, rank, world, local_rank):
                      "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
                                     if peak_kind == "measured" else "fallback 1590 TFLOP/s",
                      "algorithmic_flops_per_step": flops,
-                     "note": "the pass computes S and dP twice (7 tile products), the metric counts 5"},
+                     "note": "the pass computes S and dP twice (7 tile products), the metric counts 5" if det
+                     else "one kernel per key tile (5 tile products) plus bulk fp32 reductions of dQ"},
         "gpu_launches": 3 * args.steps,
-        "gpu_launches_note": "per step: prep, dK/dV and dQ kernels",
+        "gpu_launches_note": "per step: prep, dK/dV and dQ kernels" if det
+        else "per step: prep, the dK/dV/dQ kernel and the dQ conversion (plus a memset of the accumulator)",
         "clocks": clk,
     }
 
@@ -599,6 +605,7 @@ def main():
                     help=f"default {BENCH_WORKLOAD} ({RING_WORKLOAD} with --ring)")
     ap.add_argument("--bh", default=None, help="override B,H of the workload (profiling runs)")
     ap.add_argument("--backward", action="store_true", help="time the backward pass instead (its own JSON line)")
+    ap.add_argument("--atomic", action="store_true", help="with --backward: the non-deterministic variant")
     ap.add_argument("--ring", action="store_true", help="time ring attention of one sequence over the ranks")
     ap.add_argument("--proj", action="store_true", help="time attention + output projection (fa_fwd_proj)")
     args = ap.parse_args()

@@ -248,6 +248,29 @@ fa_status fa_fwd_noalloc(const void *q, const void *k, const void *v, void *o, f
                          fa_layout layout, int causal, float scale, fa_dtype dtype, void *stream);
 
 /*
+ * fa_bwd_atomic -- the backward pass's non-deterministic variant (page "catlass
+ * FlashAttention template tuning" (hwcomputing.csdn.net/6a0d4681), section on
+ * the backward: the `deterministic` switch, atomic adds when off).  Same
+ * arithmetic and arguments as fa_bwd, D = 128 only (else FA_ERR_UNSUPPORTED).
+ * One kernel per 128-key tile computes dK, dV and that tile's share of dQ;
+ * the shares are added into an fp32 accumulator in the workspace by bulk
+ * reductions in whatever order the tiles finish, so dq may differ between
+ * runs by fp32 rounding (dk and dv do not).  A last pass scales the
+ * accumulator and rounds it into dq.
+ *
+ * workspace   device memory of fa_bwd_atomic_workspace_size(B, H, Sq, D)
+ *             bytes, 16-byte aligned, caller-owned scratch (the per-row sums
+ *             and the dQ accumulator, zeroed here on the stream)
+ *
+ * Everything else as for fa_bwd.
+ */
+size_t fa_bwd_atomic_workspace_size(int64_t B, int64_t H, int64_t Sq, int64_t D);
+fa_status fa_bwd_atomic(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                        const float *lse, void *dq, void *dk, void *dv, int64_t B, int64_t H, int64_t Sq,
+                        int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * fa_lse_merge -- merges one partial attention result into a running one.
  * Attention over a key range split into blocks (ring / context-parallel
  * attention: page "FlashAttention in ops-transformer on Ascend NPU"

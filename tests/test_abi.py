@@ -308,3 +308,17 @@ def test_fwd_proj_host_validation(lib):
     assert call(y=Q) == fa.FA_ERR_ALIAS
     assert call(w=O) == fa.FA_ERR_ALIAS
     assert call(scale=float("inf")) == fa.FA_ERR_INVALID_ARG
+
+
+def test_bwd_atomic_workspace_and_validation(lib):
+    # the per-row sums plus a [B * H, Sq_pad, D] fp32 accumulator
+    assert fa.fa_bwd_atomic_workspace_size(1, 2, 513, 128) == 2 * 640 * (2 + 128) * 4
+    assert fa.fa_bwd_atomic_workspace_size(1, 2, 0, 128) == 0
+
+    def call(**kw):
+        a = dict(D=128, ws_bytes=fa.fa_bwd_atomic_workspace_size(1, 2, 64, 128))
+        a.update(kw)
+        return fa.fa_bwd_atomic(Q, K, V, O, DO_, L, DQ, DK, DV, 1, 2, 64, 64, a["D"], fa.FA_BSND, 1, 0.125,
+                                fa.FA_BF16, WSB, a["ws_bytes"], None)
+    assert call(D=64) == fa.FA_ERR_UNSUPPORTED
+    assert call(ws_bytes=fa.fa_bwd_workspace_size(1, 2, 64)) == fa.FA_ERR_INVALID_ARG   # too small for dQ
