@@ -43,9 +43,7 @@ constexpr int ST_EMPTY = ST_FULL + NST;
 constexpr int S_FULL = ST_EMPTY + NST;
 constexpr int DP_FULL = S_FULL + 1;
 constexpr int DQ_FULL = DP_FULL + 1;          // two: dQ^T buffer 0 / 1 complete
-constexpr int RD_A = DQ_FULL + 2;             // both groups have read S^T (256 arrivals)
-constexpr int RD_B = RD_A + 1;                // ... dP^T (256)
-constexpr int W_A = RD_B + 1;                 // P^T written (256)
+constexpr int W_A = DQ_FULL + 2;              // P^T written (256 arrivals)
 constexpr int W_B = W_A + 1;                  // dS^T written to TMEM and shared memory (256)
 constexpr int RD_C = W_B + 1;                 // two: a dQ^T buffer read (256)
 constexpr int STG_FREE = RD_C + 2;            // the staging tile may be written (1)
@@ -90,6 +88,10 @@ __device__ __forceinline__ void bulk_reduce_add_f32(void* dst, uint32_t src, uin
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// TMEM column of the 16-bit P^T / dS^T words of queries [16 kk, 16 kk + 16) of
+// a 64-query step: group g packs its 32 queries into columns [32 g, 32 g + 16).
+__device__ __forceinline__ uint32_t packed_col64(int kk) { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); }
 
 // The two 64-row boxes of one Q / dO sub-tile (rows s0 .. s0 + 63 of head h, batch b).
 __device__ __forceinline__ void load_sub(uint32_t dst, const CUtensorMap* map, uint32_t bar, int bhsd, int s0, int h,
@@ -140,8 +142,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bar(DQ_FULL + i), 1);
       mbar_init(bar(RD_C + i), 2 * BM);
     }
-    mbar_init(bar(RD_A), 2 * BM);
-    mbar_init(bar(RD_B), 2 * BM);
     mbar_init(bar(W_A), 2 * BM);
     mbar_init(bar(W_B), 2 * BM);
     mbar_init(bar(STG_FREE), 1);
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < SUB / 16; ++kk)   // dV += P^T dO_u
-          mma_ts_elect(tDV, tST + kk * 8, do_mn + (uint64_t)(kk * 128), IDESC_ACC, (u > 0 || kk > 0) ? 1u : 0u);
+          mma_ts_elect(tDV, tST + packed_col64(kk), do_mn + (uint64_t)(kk * 128), IDESC_ACC, (u > 0 || kk > 0) ? 1u : 0u);
         const bool more = u + 1 < (uint32_t)nu;
         if (more) {
           ok = wait_bar(bar(ST_FULL + (u + 1) % NST), ((u + 1) / NST) & 1u, abort_flag, limit);
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < SUB / 16; ++kk)   // dK += dS^T Q_u
-          mma_ts_elect(tDK, tDPT + kk * 8, q_mn + (uint64_t)(kk * 128), IDESC_ACC, (u > 0 || kk > 0) ? 1u : 0u);
+          mma_ts_elect(tDK, tDPT + packed_col64(kk), q_mn + (uint64_t)(kk * 128), IDESC_ACC, (u > 0 || kk > 0) ? 1u : 0u);
         tc_commit_elect(bar(ST_EMPTY + st));
         if (more) {
           kmajor_products(tDPT, dVk, do_k(u + 1));
@@ -347,12 +347,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           pk[e] = pack2<BF16>(pa, pb);
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(RD_A));
-      ok = wait_bar(bar(RD_A), u & 1u, abort_flag, limit);
-      if (!ok) break;
-      tc_fence_after();
-      tmem_st16(tST + grp * 16, pk);
+      // over the first half of this group's own S^T columns: no other thread reads them
+      tmem_st16(tST + grp * 32, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(W_A));
@@ -374,12 +370,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           pg[e] = pack2<BF16>(pp.x * (__uint_as_float(dp[2 * e]) - d2.x), pp.y * (__uint_as_float(dp[2 * e + 1]) - d2.y));
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(RD_B));
-      ok = wait_bar(bar(RD_B), u & 1u, abort_flag, limit);
-      if (!ok) break;
-      tc_fence_after();
-      tmem_st16(tDPT + grp * 16, pg);
+      tmem_st16(tDPT + grp * 32, pg);
       if (u >= 1) {                            // dQ^T(u - 1) has finished reading the shared dS^T tile
         ok = wait_bar(bar(DQ_FULL + ((u - 1) & 1u)), ((u - 1) >> 1) & 1u, abort_flag, limit);
         if (!ok) break;

@@ -19,7 +19,8 @@
 //   2. dK/dV kernel, one CTA per 128-key tile: S^T = K Q_i^T and
 //      dP^T = V dO_i^T for every visible query tile i put the keys on the TMEM
 //      lanes; two threads per key (one per half of the query columns) compute
-//      P^T and dS^T, write them (16-bit) over S^T / dP^T, and dV += P^T dO_i,
+//      P^T and dS^T, write them (16-bit) over the S^T / dP^T columns they read
+//      themselves, and dV += P^T dO_i,
 //      dK += dS^T Q_i take them as the TMEM operand -- the same MMA forms as
 //      the forward's O += P V.
 //   3. dQ kernel, one CTA per 128-query tile: S = Q K_j^T, dP = dO V_j^T,
@@ -50,8 +51,8 @@ struct Cfg {
   static constexpr int ST_EMPTY = ST_FULL + NSTAGE;
   static constexpr int S_FULL = ST_EMPTY + NSTAGE;   // S^T (dK/dV) or S and dP (dQ) of a step are in TMEM
   static constexpr int DP_FULL = S_FULL + 1;         // dP^T of a step is in TMEM (dK/dV)
-  static constexpr int RD_A = DP_FULL + 1;           // both groups have read S^T (dK/dV) or S, dP (dQ): 256 arrivals
-  static constexpr int RD_B = RD_A + 1;              // both groups have read dP^T (dK/dV): 256
+  static constexpr int RD_A = DP_FULL + 1;           // dQ: both groups have read S and dP (256 arrivals)
+  static constexpr int RD_B = RD_A + 1;              // (unused)
   static constexpr int W_A = RD_B + 1;               // P^T (dK/dV) or dS (dQ) written: 256
   static constexpr int W_B = W_A + 1;                // dS^T written (dK/dV): 256
   static constexpr int ACC_FULL = W_B + 1;           // the accumulators are final
@@ -142,6 +143,10 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, 
   for (int bx = 0; bx < nbox; ++bx)
     tma_load_4d(dst + bx * BOX_BYTES, map, bar, bx * 64, bhsd ? s0 : h, bhsd ? h : s0, b);
 }
+
+// TMEM column of the 16-bit P^T / dS^T words of queries [16 kk, 16 kk + 16) of
+// a 128-query step: group g packs its 64 queries into columns [64 g, 64 g + 32).
+__device__ __forceinline__ uint32_t packed_col(int kk) { return (uint32_t)((kk >> 2) * 64 + (kk & 3) * 8); }
 
 // ----------------------------------------------------------------------------- 2. dK, dV
 
@@ -275,7 +280,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)    // dV += P^T dO_n  (P^T: 8 packed columns per 16 queries)
-          mma_ts_elect(tDV, tST + kk * 8, do_mn + (uint64_t)(kk * 128), IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
+          mma_ts_elect(tDV, tST + packed_col(kk), do_mn + (uint64_t)(kk * 128), IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
         const bool more = n + 1 < (uint32_t)nq;
         if (more) {
           ok = wait_bar(bar(C::ST_FULL + (n + 1) % NSTAGE), ((n + 1) / NSTAGE) & 1u, abort_flag, limit);
@@ -289,7 +294,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)    // dK += dS^T Q_n
-          mma_ts_elect(tDK, tDPT + kk * 8, q_mn + (uint64_t)(kk * 128), IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
+          mma_ts_elect(tDK, tDPT + packed_col(kk), q_mn + (uint64_t)(kk * 128), IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
         tc_commit_elect(bar(C::ST_EMPTY + st));
         if (more) {
           dpt_products(n + 1);
@@ -351,14 +356,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           pk[ch * 16 + e] = pack2<BF16>(pa, pb);
         }
       }
-      // P^T of group g goes over S^T columns [32 g, 32 g + 32), which group 0
-      // reads: both groups finish reading first.
-      tc_fence_before();
-      mbar_arrive(bar(C::RD_A));
-      ok = wait_bar(bar(C::RD_A), n & 1u, abort_flag, limit);
-      if (!ok) break;
-      tc_fence_after();
-      tmem_st32(tST + grp * 32, pk);
+      // P^T of group g goes over the first half of the S^T columns it read
+      // itself, [64 g, 64 g + 32): no other thread reads them.
+      tmem_st32(tST + grp * 64, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::W_A));
@@ -383,12 +383,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           pg[ch * 16 + e] = pack2<BF16>(pp.x * (__uint_as_float(dp[2 * e]) - da), pp.y * (__uint_as_float(dp[2 * e + 1]) - db));
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(C::RD_B));
-      ok = wait_bar(bar(C::RD_B), n & 1u, abort_flag, limit);
-      if (!ok) break;
-      tc_fence_after();
-      tmem_st32(tDPT + grp * 32, pg);
+      tmem_st32(tDPT + grp * 64, pg);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::W_B));
@@ -574,7 +569,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t tS = s_buf(j);
 #pragma unroll
       for (int kk = 0; kk < BN / 16; ++kk)    // dQ += dS K_j
-        mma_ts_elect(tDQ, tS + kk * 8, k_mn + (uint64_t)(kk * 128), IDESC_ACC, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_ts_elect(tDQ, tS + packed_col(kk), k_mn + (uint64_t)(kk * 128), IDESC_ACC, (j > 0 || kk > 0) ? 1u : 0u);
       tc_commit_elect(bar(C::ST_EMPTY + st));
     }
     if (ok) tc_commit_elect(bar(C::ACC_FULL));
@@ -626,12 +621,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         pd[e] = pack2<BF16>(pa * (__uint_as_float(dp[2 * e]) - dsum), pb * (__uint_as_float(dp[2 * e + 1]) - dsum));
       }
-      // dS of group g goes over S columns [32 g, 32 g + 32), which group 0
-      // reads: every thread has read (the barrier above), so write now.
-      ok = wait_bar(bar(C::RD_A), (uint32_t)j & 1u, abort_flag, limit);
-      if (!ok) break;
-      tc_fence_after();
-      tmem_st32(tS + grp * 32, pd);
+      // dS of group g goes over the first half of the S columns it read
+      // itself, [64 g, 64 g + 32): no other thread reads them.
+      tmem_st32(tS + grp * 64, pd);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::W_A));
