@@ -18,11 +18,13 @@
 //                                           is written there by the compute warps)
 // TMEM: dV [0,128) | dK [128,256) | S^T [256,320) | dP^T [320,384) |
 // dQ^T [384,448) and [448,512) (two buffers).  The compute warps read each
-// dQ_u^T tile (lanes = head-dim index), stage it in shared memory as 64 rows x
-// 128 fp32 and add it to the fp32 accumulator in global memory with one bulk
-// reduction (cp.reduce.async.bulk .add.f32, 32 KB).  A last kernel scales the
-// accumulator and rounds it into dq.  The 64-query step keeps the TMEM budget
-// at 512 columns; the stream of Q / dO sub-tiles has three stages.
+// dQ_u^T tile (lanes = head-dim index) and add it to the fp32 accumulator in
+// global memory with red.global.add.f32 from registers: one warp instruction
+// covers 128 contiguous bytes of a query row.  (Staging the tile in shared
+// memory for one 32 KB bulk reduction was 12 % slower: two more barriers, a
+// proxy fence and one thread issuing.)  A last kernel scales the accumulator
+// and rounds it into dq.  The 64-query step keeps the TMEM budget at 512
+// columns; the stream of Q / dO sub-tiles has three stages.
 
 namespace fa {
 namespace bwda {
@@ -46,16 +48,13 @@ constexpr int DQ_FULL = DP_FULL + 1;          // two: dQ^T buffer 0 / 1 complete
 constexpr int W_A = DQ_FULL + 2;              // P^T written (256 arrivals)
 constexpr int W_B = W_A + 1;                  // dS^T written to TMEM and shared memory (256)
 constexpr int RD_C = W_B + 1;                 // two: a dQ^T buffer read (256)
-constexpr int STG_FREE = RD_C + 2;            // the staging tile may be written (1)
-constexpr int STG_FULL = STG_FREE + 1;        // the staging tile is written (256)
-constexpr int ACC_FULL = STG_FULL + 1;
+constexpr int ACC_FULL = RD_C + 2;
 constexpr int DRAIN = ACC_FULL + 1;
 constexpr int NBAR = DRAIN + 1;
 constexpr int SMEM_FIX = 0;                               // K tile, V tile
 constexpr int SMEM_STREAM = 2 * TILE;                     // per stage: Q_u, dO_u sub-tiles
 constexpr int SMEM_DST = SMEM_STREAM + NST * 2 * SUBT;    // dS^T: 128 keys x 64 queries, 16-bit, swizzled
-constexpr int SMEM_STG = SMEM_DST + BM * SUB * 2;         // dQ^T staging: 64 queries x 128 fp32
-constexpr int SMEM_VEC = SMEM_STG + SUB * DH * 4;         // per stage: lse2[64], dsum[64]
+constexpr int SMEM_VEC = SMEM_DST + BM * SUB * 2;         // per stage: lse2[64], dsum[64]
 constexpr int SMEM_BAR = SMEM_VEC + NST * 2 * SUB * 4;
 constexpr int SMEM_MISC = SMEM_BAR + NBAR * 8;
 constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;
@@ -79,16 +78,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
-__device__ __forceinline__ void bulk_reduce_add_f32(void* dst, uint32_t src, uint32_t bytes) {
-  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
-                   reinterpret_cast<uint64_t>(dst)),
-               "r"(src), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
 // TMEM column of the 16-bit P^T / dS^T words of queries [16 kk, 16 kk + 16) of
 // a 64-query step: group g packs its 32 queries into columns [32 g, 32 g + 16).
 __device__ __forceinline__ uint32_t packed_col64(int kk) { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); }
@@ -111,7 +100,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t sFix = smem_u32(smem + SMEM_FIX);
   const uint32_t sStr = smem_u32(smem + SMEM_STREAM);
   const uint32_t sDst = smem_u32(smem + SMEM_DST);
-  const uint32_t sStg = smem_u32(smem + SMEM_STG);
   const float* sVec = reinterpret_cast<const float*>(smem + SMEM_VEC);
   const uint32_t bars = smem_u32(smem + SMEM_BAR);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SMEM_MISC);
@@ -144,8 +132,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(bar(W_A), 2 * BM);
     mbar_init(bar(W_B), 2 * BM);
-    mbar_init(bar(STG_FREE), 1);
-    mbar_init(bar(STG_FULL), 2 * BM);
     mbar_init(bar(ACC_FULL), 1);
     mbar_init(bar(DRAIN), 1);
     *abort_flag = 0;
@@ -279,16 +265,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tST = tmem + lane_bits + COL_ST, tDPT = tmem + lane_bits + COL_DPT;
     const uint32_t tDV = tmem + lane_bits + COL_DV, tDK = tmem + lane_bits + COL_DK;
     const float c = p.scale_log2;
-    const bool leader = threadIdx.x == 0;
     float* dq_acc_bh = p.dq_acc + (size_t)bh * p.Sq_pad * DH;
     bool ok = true;
-    // phase C of step v: dQ^T(v) -> staging -> one bulk reduction into the accumulator
+    // phase C of step v: thread rit adds column rit of dQ_v (its 32 queries) to the
+    // accumulator; a warp's add covers 128 contiguous bytes of one query row
     auto phase_c = [&](uint32_t v) -> bool {
-      if (leader) {
-        bulk_wait_read0();                     // the previous reduction has read the staging tile
-        mbar_arrive(bar(STG_FREE));
-      }
-      if (!wait_bar(bar(STG_FREE), v & 1u, abort_flag, limit)) return false;
       if (!wait_bar(bar(DQ_FULL + (v & 1u)), (v >> 1) & 1u, abort_flag, limit)) return false;
       tc_fence_after();
       uint32_t r[32];
@@ -297,23 +278,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       reg_fence(r);
       tc_fence_before();
       mbar_arrive(bar(RD_C + (v & 1u)));
-      // staging [64 queries][128] fp32: this thread's head-dim index is rit
-      float* stg = reinterpret_cast<float*>(smem + SMEM_STG);
+      float* dst = dq_acc_bh + ((size_t)(u_begin + (int)v) * SUB + grp * 32) * DH + rit;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) stg[(grp * 32 + j) * DH + rit] = __uint_as_float(r[j]);
-      fence_proxy_async_smem();
-      mbar_arrive(bar(STG_FULL));
-      bool lok = true;
-      if (leader) {
-        lok = wait_bar1(bar(STG_FULL), v & 1u, abort_flag, limit);
-        if (lok) {
-          const int q0 = (u_begin + (int)v) * SUB;
-          bulk_reduce_add_f32(dq_acc_bh + (size_t)q0 * DH, sStg, SUB * DH * 4);
-          bulk_commit();
-        }
-      }
-      if (warp == 0) lok = __shfl_sync(0xffffffffu, lok, 0);   // keep the warp's result uniform
-      return lok;
+      for (int j = 0; j < 32; ++j) atomicAdd(dst + (size_t)j * DH, __uint_as_float(r[j]));
+      return true;
     };
     for (uint32_t u = 0; u < (uint32_t)nu && ok; ++u) {
       const uint32_t st = u % NST;
@@ -395,7 +363,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
     if (ok && nu > 0) ok = phase_c((uint32_t)nu - 1);
-    if (leader) bulk_wait0();                  // every reduction issued has completed
     // ---------------------------------------------------------------- epilogue: dV and scale * dK rows
     const bool store = key < p.Sk;
     uint8_t* dvrow = p.dv + (size_t)b * p.k_bs + (size_t)h * p.k_hs + (size_t)key * p.k_rs;

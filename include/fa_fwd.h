@@ -253,9 +253,9 @@ fa_status fa_fwd_noalloc(const void *q, const void *k, const void *v, void *o, f
  * the backward: the `deterministic` switch, atomic adds when off).  Same
  * arithmetic and arguments as fa_bwd, D = 128 only (else FA_ERR_UNSUPPORTED).
  * One kernel per 128-key tile computes dK, dV and that tile's share of dQ;
- * the shares are added into an fp32 accumulator in the workspace by bulk
- * reductions in whatever order the tiles finish, so dq may differ between
- * runs by fp32 rounding (dk and dv do not).  A last pass scales the
+ * the shares are added into an fp32 accumulator in the workspace by atomic
+ * adds in whatever order the tiles finish, so dq may differ between runs by
+ * fp32 rounding (dk and dv do not).  A last pass scales the
  * accumulator and rounds it into dq.
  *
  * workspace   device memory of fa_bwd_atomic_workspace_size(B, H, Sq, D)
