@@ -18,26 +18,31 @@
 // stream; its A tiles are read straight from the attention's output through
 // the same 4-D tensor map (either layout, no reshape or copy), mostly from L2.
 //
-// Kernel: one CTA per SM, tiles of 128 tokens x 256 features, K in blocks of
-// 64 (one 128-byte swizzled box of O, one of W per block) through a 4-stage
-// TMA ring; the MMA warp issues M = 128, N = 256, K = 16 products into one of
-// two 256-column TMEM accumulators, so that the epilogue of a tile (4 warps,
-// one token row per thread, fp32 -> 16-bit) overlaps the next tile's loop.
+// Kernel: one CTA per SM, tiles of 256 tokens x 256 features, K in blocks of
+// 64 (two 128-row swizzled boxes of O, one 256-row box of W per block) through
+// a 3-stage TMA ring; per 16 inputs the MMA warp issues two M = 128, N = 256
+// products that share the W box, into the two halves of TMEM (tokens 0-127 and
+// 128-255).  Against a 128 x 256 tile this reads a third fewer operand bytes
+// per flop (the kernel's operands come mostly from L2, and at 128 x 256 that
+// stream was ~94 bytes per SM cycle at full MMA rate).  TMEM then holds one
+// tile, so the epilogue (8 warps: token row = TMEM lane, fp32 -> 16-bit) runs
+// between tiles.
 
 namespace fa {
 namespace proj {
 
-constexpr int TM = 128;           // tokens per tile (TMEM lanes)
-constexpr int TN = 256;           // output features per tile (TMEM columns per accumulator)
+constexpr int TM = 256;           // tokens per tile: two halves of 128 (TMEM lanes)
+constexpr int TN = 256;           // output features per tile (TMEM columns per half)
 constexpr int TK = 64;            // inputs per k-block: one 128-byte box row
-constexpr int NSTAGE = 4;
-constexpr int THREADS = 192;      // warps 0-3 epilogue, 4 loads, 5 MMA
-constexpr int LOAD_WARP = 4;
-constexpr int MMA_WARP = 5;
-constexpr int A_BYTES = TM * TK * 2;   // 16 KB
+constexpr int NSTAGE = 3;
+constexpr int THREADS = 320;      // warps 0-7 epilogue (warp w: half w / 4, lanes of quadrant w % 4), 8 loads, 9 MMA
+constexpr int LOAD_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr int A_HALF = 128 * TK * 2;   // 16 KB: one 128-token box
+constexpr int A_BYTES = 2 * A_HALF;    // 32 KB
 constexpr int B_BYTES = TN * TK * 2;   // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int FULL = 0, EMPTY = NSTAGE, ACC_FULL = 2 * NSTAGE, ACC_EMPTY = ACC_FULL + 2, DRAIN = ACC_EMPTY + 2;
+constexpr int FULL = 0, EMPTY = NSTAGE, ACC_FULL = 2 * NSTAGE, ACC_EMPTY = ACC_FULL + 1, DRAIN = ACC_EMPTY + 1;
 constexpr int NBAR = DRAIN + 1;
 constexpr int SMEM_BAR = NSTAGE * STAGE_BYTES;
 constexpr int SMEM_MISC = SMEM_BAR + NBAR * 8;
@@ -73,16 +78,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bar(FULL + s), 1);
       mbar_init(bar(EMPTY + s), 1);
     }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(bar(ACC_FULL + a), 1);
-      mbar_init(bar(ACC_EMPTY + a), 4);     // one arrival per epilogue warp
-    }
+    mbar_init(bar(ACC_FULL), 1);
+    mbar_init(bar(ACC_EMPTY), 8);         // one arrival per epilogue warp
     mbar_init(bar(DRAIN), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == MMA_WARP) {
-    tmem_alloc(smem_u32(tmem_holder), 2 * TN);
+    tmem_alloc(smem_u32(tmem_holder), 2 * TN);     // 512 columns: the two 128-token halves
     tmem_relinquish();
   }
   tc_fence_before();
@@ -113,6 +116,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           mbar_arrive_expect_tx(bar(FULL + st), STAGE_BYTES);
           const int h = kb / dbox, d0 = (kb - h * dbox) * TK;
           tma_load_4d(dst, &tmO, bar(FULL + st), d0, p.bhsd ? s0 : h, p.bhsd ? h : s0, b);
+          const int s1 = s0 + 128;            // may lie past S: the box is zero-filled
+          tma_load_4d(dst + A_HALF, &tmO, bar(FULL + st), d0, p.bhsd ? s1 : h, p.bhsd ? h : s1, b);
           tma_load_4d(dst + A_BYTES, &tmW, bar(FULL + st), kb * TK, n0, 0, 0);
         }
       }
@@ -122,45 +127,47 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else if (warp == MMA_WARP) {
     constexpr uint32_t FMT = BF16 ? 1u : 0u;
-    constexpr uint32_t IDESC = idesc_f16(TM, TN, FMT, 0);
+    constexpr uint32_t IDESC = idesc_f16(128, TN, FMT, 0);    // one 128-token half per product
     bool ok = true;
     uint32_t used = 0;
     int i = 0;
     for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++i) {
-      const uint32_t a = (uint32_t)i & 1u;
-      ok = wait_bar(bar(ACC_EMPTY + a), (((uint32_t)i >> 1) & 1u) ^ 1u, abort_flag, limit);
+      ok = wait_bar(bar(ACC_EMPTY), ((uint32_t)i & 1u) ^ 1u, abort_flag, limit);   // the last tile is read
       if (!ok) break;
       tc_fence_after();
-      const uint32_t acc = tmem + a * TN;
       for (int kb = 0; kb < p.kb; ++kb, ++used) {
         const uint32_t st = used % NSTAGE;
         ok = wait_bar(bar(FULL + st), (used / NSTAGE) & 1u, abort_flag, limit);
         if (!ok) break;
         tc_fence_after();
         const uint32_t src = sbase + st * STAGE_BYTES;
-        const uint64_t da = sdesc(src, 16, 1024), db = sdesc(src + A_BYTES, 16, 1024);
+        const uint64_t da0 = sdesc(src, 16, 1024), da1 = sdesc(src + A_HALF, 16, 1024);
+        const uint64_t db = sdesc(src + A_BYTES, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < TK / 16; ++kk)
-          mma_ss_elect(acc, da + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < TK / 16; ++kk) {
+          const uint32_t acc_in = (kb > 0 || kk > 0) ? 1u : 0u;
+          mma_ss_elect(tmem, da0 + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), IDESC, acc_in);
+          mma_ss_elect(tmem + TN, da1 + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), IDESC, acc_in);
+        }
         tc_commit_elect(bar(EMPTY + st));
       }
       if (!ok) break;
-      tc_commit_elect(bar(ACC_FULL + a));
+      tc_commit_elect(bar(ACC_FULL));
     }
     tc_commit_elect(bar(DRAIN));
     if (lane == 0) drain_wait(bar(DRAIN), 0, limit);
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue: thread = token row of the tile
-    const int row = warp * 32 + lane;
-    const uint32_t lane_bits = (uint32_t)(warp * 32) << 16;
+    const int half = warp >> 2, quad = warp & 3;
+    const int row = half * 128 + quad * 32 + lane;
+    const uint32_t lane_bits = (uint32_t)(quad * 32) << 16;
     bool ok = true;
     int i = 0;
     for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++i) {
       int b, s0, n0;
       tile_coords(t, b, s0, n0);
-      const uint32_t a = (uint32_t)i & 1u;
-      ok = wait_bar(bar(ACC_FULL + a), ((uint32_t)i >> 1) & 1u, abort_flag, limit);
+      ok = wait_bar(bar(ACC_FULL), (uint32_t)i & 1u, abort_flag, limit);
       if (!ok) break;
       tc_fence_after();
       const int s = s0 + row;
@@ -168,7 +175,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll 1
       for (int c = 0; c < TN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tmem + lane_bits + a * TN + c * 32, r);
+        tmem_ld32(tmem + lane_bits + half * TN + c * 32, r);
         tmem_wait_ld();
         reg_fence(r);
         const int n = n0 + c * 32;
@@ -187,7 +194,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(ACC_EMPTY + a));
+      if (lane == 0) mbar_arrive(bar(ACC_EMPTY));
     }
   }
 
