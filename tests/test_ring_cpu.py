@@ -193,3 +193,52 @@ def test_gloo_ring_exchange_matches_whole_attention(world, causal, layout):
     o_ref, l_ref = _oracle_whole(q, k, v, layout, causal, 0.25)
     assert float((o - o_ref).abs().max()) < 1e-12
     assert float((l - l_ref).abs().max()) < 1e-12
+
+
+def _gloo_subgroup_worker(rank, world, port, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        from attention_forward_19_b200 import ring as ring_mod
+        members = [0, 2]                       # global ranks 0 and 2 are group ranks 0 and 1
+        group = dist.new_group(members)
+        if rank in members:
+            grank = members.index(rank)
+            q, k, v = _qkv("BHSD", S=2 * 2 * 5)
+            mine = [ring_mod.shard(t, grank, 2, "BHSD") for t in (q, k, v)]
+            ex = ring_mod.P2PExchange(group)
+            assert (ex.rank, ex.world) == (grank, 2)
+            # the peers are named by their global ranks: the other member, in both directions
+            assert ex.next == ex.prev == members[1 - grank]
+            o, l = ring_mod.ring_steps(*mine, grank, 2, ex, OracleOps("BHSD", 0.25), True)
+            out[grank] = (o.numpy(), l.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gloo_ring_on_a_subgroup_maps_group_ranks_to_global_ranks():
+    world = 3
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    procs = [ctx.Process(target=_gloo_subgroup_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = dict(out)
+    o = ring.unshard([torch.from_numpy(res[r][0]) for r in range(2)], "BHSD")
+    l = ring.unshard([torch.from_numpy(res[r][1]) for r in range(2)], "BHSD", seq_dim=2)
+    q, k, v = _qkv("BHSD", S=2 * 2 * 5)
+    o_ref, l_ref = _oracle_whole(q, k, v, "BHSD", True, 0.25)
+    assert float((o - o_ref).abs().max()) < 1e-12
+    assert float((l - l_ref).abs().max()) < 1e-12
