@@ -52,8 +52,7 @@ struct Cfg {
   static constexpr int S_FULL = ST_EMPTY + NSTAGE;   // S^T (dK/dV) or S and dP (dQ) of a step are in TMEM
   static constexpr int DP_FULL = S_FULL + 1;         // dP^T of a step is in TMEM (dK/dV)
   static constexpr int RD_A = DP_FULL + 1;           // dQ: both groups have read S and dP (256 arrivals)
-  static constexpr int RD_B = RD_A + 1;              // (unused)
-  static constexpr int W_A = RD_B + 1;               // P^T (dK/dV) or dS (dQ) written: 256
+  static constexpr int W_A = RD_A + 1;               // P^T (dK/dV) or dS (dQ) written: 256
   static constexpr int W_B = W_A + 1;                // dS^T written (dK/dV): 256
   static constexpr int ACC_FULL = W_B + 1;           // the accumulators are final
   static constexpr int DRAIN = ACC_FULL + 1;
@@ -186,8 +185,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(bar(C::S_FULL), 1);
     mbar_init(bar(C::DP_FULL), 1);
-    mbar_init(bar(C::RD_A), 2 * BM);
-    mbar_init(bar(C::RD_B), 2 * BM);
     mbar_init(bar(C::W_A), 2 * BM);
     mbar_init(bar(C::W_B), 2 * BM);
     mbar_init(bar(C::ACC_FULL), 1);
@@ -476,7 +473,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(bar(C::S_FULL), 1);
     mbar_init(bar(C::DP_FULL), 1);
     mbar_init(bar(C::RD_A), 2 * BM);
-    mbar_init(bar(C::RD_B), 2 * BM);
     mbar_init(bar(C::W_A), 2 * BM);
     mbar_init(bar(C::W_B), 2 * BM);
     mbar_init(bar(C::ACC_FULL), 1);
