@@ -102,6 +102,8 @@ RING_CASES = [
     (4, "BHSD", torch.bfloat16, 1, 3, 1032, 128, True),     # chunks of 129 rows
     (4, "BSND", torch.float16, 1, 2, 2048, 128, True),
     (3, "BSND", torch.bfloat16, 1, 2, 1536, 128, False),
+    (8, "BSND", torch.float16, 1, 2, 2048, 64, False),      # 16 chunks of 128 rows
+    (8, "BHSD", torch.bfloat16, 2, 2, 1040, 128, True),     # 16 chunks of 65 rows
 ]
 
 
