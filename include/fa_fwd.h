@@ -39,6 +39,12 @@
  * softmax runs in fp32; the probabilities are rounded to the input dtype
  * before P.V (fp32 accumulation); O is rounded to the input dtype once, at
  * the end; LSE is fp32.
+ *
+ * Besides the forward pass (fa_fwd, fa_fwd_ws, fa_fwd_noalloc, fa_fwd_varlen)
+ * the library exports its backward pass (fa_bwd, fa_bwd_atomic), the merge of
+ * partial results that ring attention over several GPUs is built from
+ * (fa_lse_merge), and the attention output projection (fa_out_proj,
+ * fa_fwd_proj).  Each is described at its declaration below.
  */
 #ifndef FA_FWD_H
 #define FA_FWD_H
