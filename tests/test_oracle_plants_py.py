@@ -138,3 +138,63 @@ def test_real_projection_passes_the_pins():
 @pytest.mark.parametrize("plant", [1, 2, 3, 4])
 def test_planted_projection_mistake_fails_a_pin(plant):
     assert not _proj_pins_pass(_proj_variant(plant))
+
+
+# ----------------------------------------------------------------------------- backward
+
+
+def _bwd_variant(plant):
+    """The backward of one (batch, head) with one planted mistake (plant = 0: the oracle's own function)."""
+    from oracle import attn_bwd
+
+    if plant == 0:
+        def real(q, k, v, do, causal, scale):
+            _, _, dq, dk, dv = attn_bwd.attention_fwd_bwd(q[None, None], k[None, None], v[None, None],
+                                                          do[None, None], layout="BHSD", causal=causal, scale=scale)
+            return dq[0, 0], dk[0, 0], dv[0, 0]
+        return real
+
+    def wrong(q, k, v, do, causal, scale):
+        q, k, v, do = (t.double().numpy() for t in (q, k, v, do))
+        Sq, Sk = q.shape[0], k.shape[0]
+        s = scale * (q @ k.T)
+        if causal:
+            s = np.where(np.arange(Sk)[None, :] <= np.arange(Sq)[:, None], s, -np.inf)
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        o = p @ v
+        dv = (p @ do) if plant == 1 else (p.T @ do)             # 1: P where P^T belongs (square case)
+        dp = do @ v.T
+        d_row = (do * o).sum(axis=1, keepdims=True)
+        ds = p * dp if plant == 2 else p * (dp - d_row)           # 2: the row sum D dropped
+        dq = (ds @ k) if plant == 3 else scale * (ds @ k)         # 3: dQ without the scale
+        dk = scale * (ds @ q) if plant == 4 else scale * (ds.T @ q)   # 4: dS where dS^T belongs
+        return dq, dk, dv
+    return wrong
+
+
+def _bwd_pin_passes(bwd):
+    """Agreement with torch autograd through the textbook forward (the first pin of test_oracle_bwd.py)."""
+    g = torch.Generator().manual_seed(3)
+    S, D, scale = 9, 8, 0.43
+    q, k, v, do = (torch.randn(S, D, generator=g, dtype=torch.float64) for _ in range(4))
+    for causal in (False, True):
+        dq, dk, dv = bwd(q, k, v, do, causal, scale)
+        qt, kt, vt = (t.clone().requires_grad_(True) for t in (q, k, v))
+        s = scale * qt @ kt.T
+        if causal:
+            s = s.masked_fill(torch.triu(torch.ones(S, S, dtype=torch.bool), 1), float("-inf"))
+        (torch.softmax(s, dim=-1) @ vt * do).sum().backward()
+        for mine, ref in ((dq, qt.grad), (dk, kt.grad), (dv, vt.grad)):
+            if not np.max(np.abs(np.asarray(mine) - ref.numpy())) < 1e-10:
+                return False
+    return True
+
+
+def test_real_backward_passes_the_autograd_pin():
+    assert _bwd_pin_passes(_bwd_variant(0))
+
+
+@pytest.mark.parametrize("plant", [1, 2, 3, 4])
+def test_planted_backward_mistake_fails_the_autograd_pin(plant):
+    assert not _bwd_pin_passes(_bwd_variant(plant))
