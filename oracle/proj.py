@@ -12,7 +12,6 @@ attention, every token's head outputs concatenated head after head,
 with W in a linear layer's [E, H * D] layout.  The contraction is one numpy
 matmul on the exact fp64 decoding of the 16-bit inputs.
 """
-import numpy as np
 import torch
 
 

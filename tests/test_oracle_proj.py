@@ -4,7 +4,6 @@ Independent of the numpy matmul it uses: identity and selector weights (closed
 forms), a pure-Python loop over a tiny case, and, for the composition with
 attention, a one-key closed form.
 """
-import math
 
 import numpy as np
 import pytest
