@@ -1243,10 +1243,13 @@ struct SelfTest {
   unsigned long long wait_limit_ns;
 };
 
-fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
-                   int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
-                   unsigned int* sched, void* stream, const SelfTest* selftest = nullptr) {
-  // ---- arguments that need no device
+// Every check of a dense forward call's arguments that needs no device, in
+// the order fa_fwd applies them.  FA_OK with *noop set: the call has no query
+// rows and nothing to do (the pointers are then not looked at).
+fa_status host_checks(const void* q, const void* k, const void* v, const void* o, const float* lse, int64_t B,
+                      int64_t H, int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, float scale, fa_dtype dtype,
+                      bool* noop) {
+  *noop = false;
   if (B <= 0 || H <= 0 || Sq < 0 || Sk <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
   if (layout != FA_BSND && layout != FA_BHSD) return FA_ERR_INVALID_ARG;
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
@@ -1257,7 +1260,10 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   if (B >= lim || H >= lim || Sq >= lim || Sk >= lim || B * H >= lim) return FA_ERR_UNSUPPORTED;
   const int64_t nqb = (Sq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
   if (B * H * nqb >= lim) return FA_ERR_UNSUPPORTED;
-  if (Sq == 0) return FA_OK;
+  if (Sq == 0) {
+    *noop = true;
+    return FA_OK;
+  }
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v) |
        reinterpret_cast<uintptr_t>(o)) & 15u)
@@ -1269,6 +1275,17 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
       overlaps(lse, lbytes, q, qbytes) || overlaps(lse, lbytes, k, kvbytes) ||
       overlaps(lse, lbytes, v, kvbytes) || overlaps(lse, lbytes, o, qbytes))
     return FA_ERR_ALIAS;
+  return FA_OK;
+}
+
+fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                   int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
+                   unsigned int* sched, void* stream, const SelfTest* selftest = nullptr) {
+  // ---- arguments that need no device
+  bool noop = false;
+  fa_status hst = host_checks(q, k, v, o, lse, B, H, Sq, Sk, D, layout, scale, dtype, &noop);
+  if (hst != FA_OK || noop) return hst;
+  const int64_t nqb = (Sq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
 
   // ---- device checks
   int dev = 0, sms = 0;
@@ -1326,14 +1343,13 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
 // its device address comes from cudaGetSymbolAddress, once per device, with
 // that device current, on the first fa_fwd_noalloc call there.
 constexpr size_t kNoAllocScratchBytes = 256;   // capacity of the fixed scratch
+// The schedule needs kWorkspaceBytes whatever the call's sizes, so the fixed
+// array always suffices; a scratch need that grew with the sizes would have
+// to be refused at run time instead.
 static_assert(kWorkspaceBytes <= kNoAllocScratchBytes, "the fixed scratch cannot hold the schedule's counter");
 
-struct NoAllocScratch {
-  std::once_flag once;
-  void* ptr = nullptr;
-  int err = 0;
-};
-NoAllocScratch g_noalloc[kMaxDevices];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices];   // a device's looked-up address; null until a lookup succeeds
 
 }  // namespace
 
@@ -1341,22 +1357,25 @@ static __device__ __align__(256) unsigned char fa_noalloc_scratch[kNoAllocScratc
 
 namespace {
 
-// Device address of fa_noalloc_scratch on `dev` (the current device), looked
-// up on the first call for that device; nullptr with *err set on failure.
-void* noalloc_scratch_address(int dev, int* err) {
-  NoAllocScratch& slot = g_noalloc[dev];
-  std::call_once(slot.once, [&slot] {
+// Device address of fa_noalloc_scratch on `dev` (the current device).  Only a
+// successful lookup is kept, so a failed one (say, attempted during a stream
+// capture) is simply tried again by the next call.  `refresh` forces a new
+// lookup: after cudaDeviceReset the module is loaded anew and a kept address
+// may be stale.  nullptr with *err set on failure.
+void* noalloc_scratch_address(int dev, bool refresh, int* err) {
+  std::lock_guard<std::mutex> g(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev] || refresh) {
     void* ptr = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&ptr, fa_noalloc_scratch);
     if (e != cudaSuccess) {
       cudaGetLastError();
-      slot.err = (int)e;
-      return;
+      g_noalloc_ptr[dev] = nullptr;
+      *err = (int)e;
+      return nullptr;
     }
-    slot.ptr = ptr;
-  });
-  *err = slot.err;
-  return slot.ptr;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
 }
 
 }  // namespace
@@ -1367,22 +1386,21 @@ fa_status fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, f
                          int64_t H, int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale,
                          fa_dtype dtype, void* stream) {
   // arguments that need no device, answered exactly as fa_fwd answers them
-  if (B <= 0 || H <= 0 || Sq < 0 || Sk <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
-  if (layout != FA_BSND && layout != FA_BHSD) return FA_ERR_INVALID_ARG;
-  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
-  if (Sq == 0) return FA_OK;
-  // the schedule needs kWorkspaceBytes of scratch whatever the sizes; a need
-  // beyond the fixed array is refused rather than overrun
-  if (kWorkspaceBytes > kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;
+  bool noop = false;
+  fa_status st = host_checks(q, k, v, o, lse, B, H, Sq, Sk, D, layout, scale, dtype, &noop);
+  if (st != FA_OK || noop) return st;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail((int)e);
   if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
   int err = 0;
-  void* scratch = noalloc_scratch_address(dev, &err);
+  void* scratch = noalloc_scratch_address(dev, false, &err);
   if (!scratch) return cuda_fail(err);
+  if (check_device_ptr(scratch, dev) != FA_OK) {
+    // a kept address that no longer names device memory here: look it up once more
+    scratch = noalloc_scratch_address(dev, true, &err);
+    if (!scratch) return cuda_fail(err);
+  }
   return fwd_impl(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype,
                   static_cast<unsigned int*>(scratch), stream);
 }

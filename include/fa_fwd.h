@@ -239,15 +239,18 @@ fa_status fa_selftest_wait_timeout(const void *q, const void *k, const void *v, 
  *
  * The dynamic schedule's scratch (its work counter, 16 bytes) lives in a
  * fixed 256-byte array inside the library, held by every GPU that loads the
- * library until the process exits.  The first call on a device looks up that
- * array's device address (cudaGetSymbolAddress, with the device current);
- * make that first call before any stream capture.  Every call zeroes the
- * counter on `stream` before its launch and then uses it, so calls that
+ * library until the process exits.  The counter's size does not depend on
+ * the call's sizes, so no size is too large for the array.  The first call
+ * on a device looks up that array's device address (cudaGetSymbolAddress,
+ * with the device current); make that first call before any stream capture.
+ * Only a successful lookup is kept: a lookup that fails returns FA_ERR_CUDA
+ * and is tried again by the next call.  After cudaDeviceReset the kept
+ * address is checked, found stale and looked up again.  Every call zeroes
+ * the counter on `stream` before its launch and then uses it, so calls that
  * overlap on the same GPU (for example on two streams) race on it: serialise
  * them, or use fa_fwd_ws with separate workspaces.  Each GPU has its own copy
- * of the array.  Arguments, results and errors as for fa_fwd;
- * FA_ERR_UNSUPPORTED if the schedule ever needed more scratch than the array
- * holds.
+ * of the array.  Arguments, results and errors as for fa_fwd, checked in the
+ * same order.
  */
 fa_status fa_fwd_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
                          int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D,

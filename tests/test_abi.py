@@ -164,6 +164,36 @@ def test_dynamic_schedule_argument_errors_match_static(lib):
         assert call_ws(**kw) == call(**kw) == fa.FA_ERR_INVALID_ARG
 
 
+def call_noalloc(q=Q, k=K, v=V, o=O, lse=L, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_fwd_noalloc(q, k, v, o, lse, a["B"], a["H"], a["Sq"], a["Sk"], a["D"], a["layout"], a["causal"],
+                             a["scale"], a["dtype"], None)
+
+
+NOALLOC_CASES = [dict(B=0), dict(H=0), dict(Sk=0), dict(Sq=-1), dict(D=0), dict(layout=2), dict(dtype=2),
+                 dict(scale=float("nan")), dict(D=96), dict(D=256), dict(Sq=1 << 31), dict(Sk=1 << 31),
+                 dict(B=1 << 30, Sq=0), dict(H=1 << 30, Sq=0), dict(Sq=0), dict(Sq=0, q=0, o=0, lse=0),
+                 dict(q=0), dict(lse=0), dict(q=Q + 8), dict(o=O + 8), dict(lse=L + 2), dict(o=Q),
+                 dict(o=O, lse=O + 16), dict(lse=V + 64)]
+
+
+@pytest.mark.parametrize("kw", NOALLOC_CASES, ids=lambda kw: ",".join(f"{k}={v}" for k, v in kw.items()))
+def test_noalloc_argument_errors_match_fa_fwd(lib, kw):
+    """fa_fwd_noalloc answers every call that fails before the device exactly as fa_fwd does,
+    in the same order (a size beyond the limits is refused even when Sq = 0)."""
+    assert call_noalloc(**kw) == call(**kw)
+
+
+def test_noalloc_reaches_device_checks(lib):
+    # valid arguments: the call gets past the host checks to the device lookup, which fails on a
+    # machine without a GPU (FA_ERR_CUDA) or on the fake pointers (FA_ERR_NOT_DEVICE_POINTER / CUDA)
+    st = call_noalloc()
+    assert st not in (fa.FA_OK, fa.FA_ERR_INVALID_ARG, fa.FA_ERR_MISALIGNED, fa.FA_ERR_ALIAS,
+                      fa.FA_ERR_UNSUPPORTED), st
+    assert call_noalloc(B=1 << 30, Sq=0) == fa.FA_ERR_UNSUPPORTED
+
+
 def call_selftest(limit_us=20000, **kw):
     a = dict(GOOD)
     a.update(kw)

@@ -7,12 +7,16 @@ fa_fwd_noalloc serves them by keeping the dynamic schedule's scratch in a
 fixed array inside the library.  This test calls it through the C ABI, twice
 in a row (the second call must not be disturbed by what the first left in the
 shared scratch), and checks each result against fa_fwd_ws with a
-caller-provided workspace, within the tolerances of the parity tests.
+caller-provided workspace.  Both run the same kernel with the same work
+units, and a unit's result does not depend on which CTA computes it, so the
+outputs must be bit-identical; the tolerances of the parity tests, and one
+direct comparison with the fp64 oracle, are checked as well.
 
 The file is named so that pytest collects it last.
 """
 import math
 
+import numpy as np
 import pytest
 import torch
 
@@ -59,3 +63,25 @@ def test_no_alloc_entry_matches_workspace_entry(w):
         assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
         assert (o.float() - o_ref.float()).abs().max().item() <= O_TOL[w.dtype]
         assert (lse - l_ref).abs().max().item() <= LSE_TOL
+        # the same kernel and the same units: the same bits
+        assert torch.equal(o, o_ref)
+        assert torch.equal(lse, l_ref)
+
+
+def test_no_alloc_entry_against_oracle():
+    """One element-by-element comparison of fa_fwd_noalloc's output with the fp64 oracle."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from oracle import attn
+    w = Workload("noalloc_bf16_bsnd_causal_small", "bf16", "BSND", 1, 3, 700, 700, 128, True,
+                 1 / math.sqrt(128), seed=13)
+    q, k, v = make_qkv(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o, lse = torch.empty_like(qd), torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    assert _raw_call(fa.fa_fwd_noalloc, w, qd, kd, vd, o, lse, stream) == fa.FA_OK
+    assert fa.fa_device_status(stream) == fa.FA_OK
+    o_ref, lse_ref = attn.default().fwd(q, k, v, layout=w.layout, causal=w.causal, scale=float(np.float32(w.scale)))
+    o_gpu = o.cpu().permute(0, 2, 1, 3).to(torch.float64).numpy()
+    assert np.max(np.abs(o_gpu - o_ref)) <= O_TOL[w.dtype]
+    assert np.max(np.abs(lse.cpu().to(torch.float64).numpy() - lse_ref)) <= LSE_TOL
