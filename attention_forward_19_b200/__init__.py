@@ -39,7 +39,8 @@ FA_MERGE_FINAL = 2
 LAYOUTS = {"BSND": FA_BSND, "BHSD": FA_BHSD}
 
 # Names every public symbol of include/fa_fwd.h.
-EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_noalloc", "fa_fwd_varlen", "fa_bwd",
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_heads", "fa_fwd_noalloc", "fa_fwd_varlen",
+                    "fa_bwd",
                     "fa_bwd_workspace_size", "fa_bwd_atomic",
                     "fa_bwd_atomic_workspace_size", "fa_lse_merge", "fa_out_proj", "fa_fwd_proj",
                     "fa_selftest_wait_timeout", "fa_device_status", "fa_query_support", "fa_status_string",
@@ -83,6 +84,9 @@ def load_library(path=None, rebuild_if_stale=True):
     lib.fa_fwd_ws.restype = c_int
     lib.fa_fwd_ws.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, vp,
                               ctypes.c_size_t, vp]
+    lib.fa_fwd_heads.restype = c_int
+    lib.fa_fwd_heads.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, i64, i64,
+                                 vp, ctypes.c_size_t, vp]
     lib.fa_fwd_noalloc.restype = c_int
     lib.fa_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, vp]
     lib.fa_fwd_varlen.restype = c_int
@@ -139,6 +143,16 @@ def fa_fwd_ws(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, wo
     lib = load_library()
     return lib.fa_fwd_ws(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
                          int(bool(causal)), float(scale), int(dtype), workspace, int(workspace_bytes), stream)
+
+
+def fa_fwd_heads(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, head_begin, head_count,
+                 workspace, workspace_bytes, stream):
+    """The C fa_fwd_heads (only the flattened heads [head_begin, head_begin + head_count) of the
+    whole problem's tensors) with raw pointers and sizes; returns the fa_status code."""
+    lib = load_library()
+    return lib.fa_fwd_heads(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
+                            int(bool(causal)), float(scale), int(dtype), int(head_begin), int(head_count), workspace,
+                            int(workspace_bytes), stream)
 
 
 def fa_fwd_noalloc(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, stream):
@@ -267,7 +281,7 @@ def _dims(q, k, layout, head_num=None):
 
 
 def flash_attention_forward(q, k, v, layout="BSND", causal=False, scale=None, head_num=None,
-                            out=None, lse=None, stream=None, schedule="dynamic", workspace=None):
+                            out=None, lse=None, stream=None, schedule="dynamic", workspace=None, heads=None):
     """Attention forward on CUDA tensors through the C ABI.
 
     q: [B, Sq, H, D] (BSND) or [B, H, Sq, D] (BHSD); k, v likewise with Sk.
@@ -277,6 +291,9 @@ def flash_attention_forward(q, k, v, layout="BSND", causal=False, scale=None, he
     schedule="dynamic" calls fa_fwd_ws (work units handed out from a counter
     in `workspace`, a uint8 CUDA tensor of fa_fwd_workspace_size() bytes,
     allocated here when not given); "static" calls fa_fwd (no workspace).
+    heads=(head_begin, head_count) calls fa_fwd_heads instead: only the
+    flattened heads b * H + h in that range are computed, in place in the
+    whole tensors; the other heads' rows of out and lse are left as they were.
     """
     import torch
     lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
@@ -302,6 +319,23 @@ def flash_attention_forward(q, k, v, layout="BSND", causal=False, scale=None, he
     if stream is None:
         stream = torch.cuda.current_stream(q.device) if q.is_cuda else None
     sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    if heads is not None:
+        h0, hc = (int(x) for x in heads)
+        wptr, wbytes = None, 0
+        if schedule == "dynamic":
+            nbytes = fa_fwd_workspace_size()
+            if workspace is None:
+                workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+            if workspace.numel() * workspace.element_size() < nbytes or not workspace.is_contiguous():
+                raise ValueError(f"workspace must be a contiguous tensor of at least {nbytes} bytes")
+            wptr, wbytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+        elif schedule != "static":
+            raise ValueError(f"schedule must be 'dynamic' or 'static', not {schedule!r}")
+        st = fa_fwd_heads(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                          B, H, Sq, Sk, D, lay, causal, scale, dt, h0, hc, wptr, wbytes, sptr)
+        if st != FA_OK:
+            raise FaError(st, "fa_fwd_heads")
+        return out, lse
     if schedule == "static":
         st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                     B, H, Sq, Sk, D, lay, causal, scale, dt, sptr)

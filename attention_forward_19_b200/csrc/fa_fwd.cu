@@ -78,7 +78,16 @@ constexpr int UQ_CONSUMERS = 9;       // arrivals that free a unit-id slot: the 
 #endif
 constexpr float RESCALE_LOG2 = FA_RESCALE_LOG2;  // O / l are rescaled only when a row max grows by more (log2 units)
 constexpr float RESCALE_POW2 = (float)(1u << (int)FA_RESCALE_LOG2);  // 2^RESCALE_LOG2
-constexpr float HEADROOM_LOG2 = 8.0f;  // bf16 only: a moved reference sits this far above the tile max
+#ifndef FA_HEADROOM_LOG2
+#define FA_HEADROOM_LOG2 8.0f
+#endif
+constexpr float HEADROOM_LOG2 = FA_HEADROOM_LOG2;  // bf16 only: a moved reference sits this far above the tile max
+// Test builds only (FA_COUNT_BRANCHES=1): per-warp counts of the softmax's
+// rarely taken branches, read back by fa_debug_branch_counts.  The product
+// build has neither the counters nor the entry point.
+#ifndef FA_COUNT_BRANCHES
+#define FA_COUNT_BRANCHES 0
+#endif
 #ifndef FA_EMU_PAIRS
 #define FA_EMU_PAIRS 0
 #endif
@@ -123,7 +132,8 @@ struct Params {
   int B, H, Sq, Sk;      // variable-length batch: Sq, Sk = the longest sequence
   int nqb;             // query units per head: ceil(Sq / 256)
   int tk;              // key tiles: ceil(Sk / 128)
-  int bh;              // B * H
+  int bh;              // heads this launch computes (B * H, or a range of them)
+  int head0;           // first head of the range: flattened index b * H + h
   int group_heads;     // heads per L2 group of the schedule
   int total_units;     // bh * nqb
   int causal;
@@ -143,6 +153,13 @@ struct Params {
 // Device error word: bit 0 a wait ran out (FA_ERR_TIMEOUT), bit 1 invalid
 // sequence offsets of a variable-length batch (FA_ERR_INVALID_ARG).
 __device__ int g_dev_error = 0;
+
+#if FA_COUNT_BRANCHES
+// [0] warp-tiles after a unit's first tile, [1] of them with the speculative
+// pass rejected (exact recompute), [2] with O rescaled, [3] accepted with a
+// weight above 2^(RESCALE_LOG2 - 1) (a stale reference close to its bound).
+__device__ unsigned long long g_branch_counts[4];
+#endif
 
 // ----------------------------------------------------------------------------- PTX helpers
 
@@ -586,7 +603,7 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
   const int r = u - g * per_group;
   const int gs = min(p.group_heads, p.bh - g * p.group_heads);
   const int level = r / gs;
-  const int bh = g * p.group_heads + (r - level * gs);
+  const int bh = p.head0 + g * p.group_heads + (r - level * gs);
   const int qblk = p.causal ? (p.nqb - 1 - level) : level;
   Unit un;
   un.b = bh / p.H;
@@ -967,6 +984,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float corr = round_to_input<BF16>(p_top) - p_top;
         l = l * alpha + rowsum;
         ln = ln * alpha + rowsum + corr;
+#if FA_COUNT_BRANCHES
+        if (j > 0) {
+          const bool any_grow = __any_sync(0xffffffffu, grow);
+          const bool near = __any_sync(0xffffffffu, !exact && p_top > 0.5f * RESCALE_POW2);
+          if (lane == 0) {
+            atomicAdd(&g_branch_counts[0], 1ull);
+            if (exact) atomicAdd(&g_branch_counts[1], 1ull);
+            if (any_grow) atomicAdd(&g_branch_counts[2], 1ull);
+            if (near) atomicAdd(&g_branch_counts[3], 1ull);
+          }
+        }
+#endif
         if (j > 0 && __any_sync(0xffffffffu, grow)) {
           uint32_t orow[D];
           tmem_ld_cols<D / 32>(tO, orow);
@@ -1278,14 +1307,20 @@ fa_status host_checks(const void* q, const void* k, const void* v, const void* o
   return FA_OK;
 }
 
+// head_begin / head_count: the flattened heads b * H + h the launch computes
+// (all of them: 0 / -1); the tensors are the whole [B, H] problem either way.
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
                    int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
-                   unsigned int* sched, void* stream, const SelfTest* selftest = nullptr) {
+                   unsigned int* sched, void* stream, const SelfTest* selftest = nullptr, int64_t head_begin = 0,
+                   int64_t head_count = -1) {
   // ---- arguments that need no device
   bool noop = false;
   fa_status hst = host_checks(q, k, v, o, lse, B, H, Sq, Sk, D, layout, scale, dtype, &noop);
   if (hst != FA_OK || noop) return hst;
   const int64_t nqb = (Sq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+  if (head_count < 0) head_count = B * H;
+  if (head_begin < 0 || head_begin > B * H || head_count > B * H - head_begin) return FA_ERR_INVALID_ARG;
+  if (head_count == 0) return FA_OK;
 
   // ---- device checks
   int dev = 0, sms = 0;
@@ -1314,9 +1349,10 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   prm.Sk = (int)Sk;
   prm.nqb = (int)nqb;
   prm.tk = (int)((Sk + fa::BN - 1) / fa::BN);
-  prm.bh = (int)(B * H);
-  prm.group_heads = l2_group_heads(Sk, D, B * H);
-  prm.total_units = (int)(B * H * nqb);
+  prm.bh = (int)head_count;
+  prm.head0 = (int)head_begin;
+  prm.group_heads = l2_group_heads(Sk, D, head_count);
+  prm.total_units = (int)(head_count * nqb);
   prm.causal = causal ? 1 : 0;
   prm.bhsd = layout == FA_BHSD ? 1 : 0;
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634074);
@@ -1435,6 +1471,29 @@ fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float*
 
 size_t fa_fwd_workspace_size(void) { return kWorkspaceBytes; }
 
+fa_status fa_fwd_heads(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                       int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
+                       int64_t head_begin, int64_t head_count, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  if (head_begin < 0 || head_count < 0) return FA_ERR_INVALID_ARG;
+  if (B > 0 && H > 0 && (head_begin > B * H || head_count > B * H - head_begin)) return FA_ERR_INVALID_ARG;
+  if (!workspace)
+    return fwd_impl(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, nullptr, stream, nullptr,
+                    head_begin, head_count);
+  if (workspace_bytes < kWorkspaceBytes) return FA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) & 15u) return FA_ERR_MISALIGNED;
+  if (B > 0 && H > 0 && D > 0 && Sq > 0 && Sk > 0) {
+    const size_t qbytes = (size_t)(B * H * Sq * D) * 2, kvbytes = (size_t)(B * H * Sk * D) * 2;
+    const size_t lbytes = (size_t)(B * H * Sq) * 4;
+    if ((q && overlaps(workspace, workspace_bytes, q, qbytes)) || (k && overlaps(workspace, workspace_bytes, k, kvbytes)) ||
+        (v && overlaps(workspace, workspace_bytes, v, kvbytes)) || (o && overlaps(workspace, workspace_bytes, o, qbytes)) ||
+        (lse && overlaps(workspace, workspace_bytes, lse, lbytes)))
+      return FA_ERR_ALIAS;
+  }
+  return fwd_impl(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype,
+                  static_cast<unsigned int*>(workspace), stream, nullptr, head_begin, head_count);
+}
+
 fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
                         const int32_t* cu_seqlens_k, int64_t B, int64_t H, int64_t total_q, int64_t total_k,
                         int64_t max_seqlen_q, int64_t max_seqlen_k, int64_t D, int causal, float scale,
@@ -1506,6 +1565,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
   prm.nqb = (int)nqb;
   prm.tk = (int)((max_seqlen_k + fa::BN - 1) / fa::BN);
   prm.bh = (int)(B * H);
+  prm.head0 = 0;
   prm.group_heads = l2_group_heads(max_seqlen_k, D, B * H);
   prm.total_units = (int)(B * H * nqb);
   prm.causal = causal ? 1 : 0;
@@ -1538,6 +1598,18 @@ fa_status fa_device_status(void* stream) {
   }
   return FA_OK;
 }
+
+#if FA_COUNT_BRANCHES
+// Test builds only: copies the four branch counters of the current device
+// (see g_branch_counts) to out[0..3] and zeroes them.  Synchronises the device.
+int fa_debug_branch_counts(unsigned long long* out) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(out, fa::g_branch_counts, 4 * sizeof(unsigned long long));
+  const unsigned long long zero[4] = {0ull, 0ull, 0ull, 0ull};
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(fa::g_branch_counts, zero, sizeof(zero));
+  return (int)e;
+}
+#endif
 
 fa_status fa_query_support(int64_t D, fa_dtype dtype) {
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_UNSUPPORTED;

@@ -7,9 +7,14 @@ bf16 BHSD B=2 H=40 Sq=Sk=8192 D=128, causal, scale 1/sqrt(128), q/k/v ~ N(0,1).
 The metric is attention-forward TFLOP/s with the causal-halved flop count
 4*B*H*Sq*Sk*D/2.  Timing: W untimed warm-up steps, then exactly K steps
 between a barrier + torch.cuda.synchronize() on both sides, timed with CUDA
-events on the stream the kernel is launched on; with N > 1 ranks (torchrun)
-every rank processes its own full workload (weak scaling, no collective on
-the data path) and the time is the max over ranks.  The inputs (3 x 168 MB)
+events on the stream the kernel is launched on.  With N > 1 ranks (torchrun)
+the heads of one problem are split into contiguous ranges of equal work
+(attention_forward_19_b200.shard), and each rank computes its range with
+fa_fwd_heads in place; there is no collective on the data path, and the time
+is the max over ranks.  By default the problem is the workload repeated once
+per rank along the batch axis, so each rank's share is one workload (weak
+scaling); --strong splits the workload itself.  --allgather adds an all-gather
+of every rank's O/LSE rows to each step.  The inputs (3 x 168 MB per workload)
 are larger than the 126 MB L2, so no flush is done between steps.
 
 --impl reference runs the fp64 CPU oracle (the parity reference) on rank 0
@@ -200,6 +205,39 @@ def rank_workload(w0, rank):
     return w0.with_(seed=w0.seed + 1000 * rank)
 
 
+def shard_plan(w0, world, strong):
+    """The problem the ranks share and each rank's (head_begin, head_count).
+
+    Weak scaling (default): the problem is the workload repeated along the batch
+    axis once per rank (B = world * B0), so each rank's balanced share is one
+    workload's worth of heads.  Strong scaling: the problem is the workload
+    itself, split into balanced head ranges."""
+    from attention_forward_19_b200 import shard
+    wg = w0 if strong or world == 1 else w0.with_(B=w0.B * world, name=f"{w0.name}_x{world}")
+    ranges = shard.head_ranges(wg.B, wg.H, wg.Sq, wg.Sk, wg.causal, world)
+    return wg, ranges
+
+
+def rank_inputs(w0, wg, rank, world, strong, device):
+    """q, k, v of the shared problem on this rank, in the whole problem's shape.
+
+    Strong scaling: every rank holds the same whole problem (one seed).  Weak
+    scaling: rank r draws its own batches [r B0, (r + 1) B0) -- exactly its head
+    range -- from its own seed (rank_workload); the other batches stay zero and
+    are never read by this rank."""
+    if strong or world == 1:
+        return make_qkv(wg, device=device)
+    from fa_inputs import DTYPES
+    dt = DTYPES[wg.dtype]
+    q = torch.zeros(wg.q_shape(), dtype=dt, device=device)
+    k = torch.zeros(wg.kv_shape(), dtype=dt, device=device)
+    v = torch.zeros(wg.kv_shape(), dtype=dt, device=device)
+    mine = slice(rank * w0.B, (rank + 1) * w0.B)
+    for dst, src in zip((q, k, v), make_qkv(rank_workload(w0, rank), device=device)):
+        dst[mine].copy_(src)
+    return q, k, v
+
+
 def max_over_ranks(ms, world, device):
     """The slowest rank's time (a scalar all-reduce; no data-path collective)."""
     if world == 1:
@@ -211,20 +249,25 @@ def max_over_ranks(ms, world, device):
 
 def run_native(args, rank, world, local_rank):
     import attention_forward_19_b200 as fa
+    from attention_forward_19_b200 import shard
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w0 = bench_workload(args)
-    w = rank_workload(w0, rank)
-    q, k, v = make_qkv(w, device=dev)
-    o = torch.empty_like(q)
-    lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
-    # work counter of the dynamic schedule (fa_fwd_ws); zeroed by the library before every launch
+    wg, ranges = shard_plan(w0, world, args.strong)
+    h0, hc = ranges[rank]
+    q, k, v = rank_inputs(w0, wg, rank, world, args.strong, dev)
+    o = torch.zeros_like(q)
+    lse = torch.zeros((wg.B, wg.H, wg.Sq), dtype=torch.float32, device=dev)
+    # work counter of the dynamic schedule (fa_fwd_heads with a workspace); zeroed by the library
+    # before every launch
     ws = torch.empty(fa.fa_fwd_workspace_size(), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        fa.flash_attention_forward(q, k, v, layout=w.layout, causal=w.causal, scale=w.scale, out=o, lse=lse,
-                                   stream=stream, schedule="dynamic", workspace=ws)
+        fa.flash_attention_forward(q, k, v, layout=wg.layout, causal=wg.causal, scale=wg.scale, out=o, lse=lse,
+                                   stream=stream, schedule="dynamic", workspace=ws, heads=(h0, hc))
+        if args.allgather and world > 1:
+            shard.all_gather_heads(o, lse, ranges, wg.layout)
 
     for _ in range(args.warmup):
         step()
@@ -253,27 +296,31 @@ def run_native(args, rank, world, local_rank):
     fa.check_device_status(stream)
     ms_total = max_over_ranks(ms_local, world, dev)
     ms_step = ms_total / args.steps
-    flops = w.flops()
-    value = world * flops * args.steps / (ms_total * 1e-3) / 1e12
+    flops_rank = shard.flops_of_heads(hc, wg.Sq, wg.Sk, wg.D, wg.causal)
+    flops = shard.flops_of_heads(wg.B * wg.H, wg.Sq, wg.Sk, wg.D, wg.causal)   # all ranks together
+    value = flops * args.steps / (ms_total * 1e-3) / 1e12
 
     if args.no_e2e:
         if rank == 0:
-            print(f"{w.name}: {ms_step:.4f} ms/step, {value:.1f} TFLOP/s (no e2e, no baseline)", flush=True)
+            print(f"{wg.name}: {ms_step:.4f} ms/step, {value:.1f} TFLOP/s (no e2e, no baseline)", flush=True)
         return None
-    # end to end through the public API: pinned host inputs -> device -> kernel -> host result
+    # end to end through the public API: this rank's input rows from pinned host memory -> device ->
+    # kernel -> this rank's result rows (with --allgather, the whole result) back to pinned host memory
     e2e_steps = max(3, min(args.steps, 10))
-    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
-    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    dev_in = [view for t in (q, k, v) for view in shard.head_rows(t, h0, hc, wg.layout, wg.H)]
+    host_in = [view.cpu().pin_memory() for view in dev_in]
+    if args.allgather and world > 1:
+        dev_out = [o, lse]
+    else:
+        dev_out = [view for t in (o, lse) for view in shard.head_rows(t, h0, hc, wg.layout, wg.H)]
+    host_out = [torch.empty(view.shape, dtype=view.dtype, pin_memory=True) for view in dev_out]
 
     def e2e_step():
-        dq = hq.to(dev, non_blocking=True)
-        dk = hk.to(dev, non_blocking=True)
-        dv = hv.to(dev, non_blocking=True)
-        do, dl = fa.flash_attention_forward(dq, dk, dv, layout=w.layout, causal=w.causal, scale=w.scale,
-                                            stream=stream, schedule="dynamic", workspace=ws)
-        ho.copy_(do, non_blocking=True)
-        hl.copy_(dl, non_blocking=True)
+        for dst, src in zip(dev_in, host_in):
+            dst.copy_(src, non_blocking=True)
+        step()
+        for dst, src in zip(host_out, dev_out):
+            dst.copy_(src, non_blocking=True)
 
     e2e_step()
     barrier()
@@ -288,15 +335,15 @@ def run_native(args, rank, world, local_rank):
     barrier()
     e2e_ms = max_over_ranks(a0.elapsed_time(a1), world, dev)
     fa.check_device_status(stream)
-    e2e_value = world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    e2e_value = flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
 
     if rank != 0:
         return None
     peaks, peak_kind = load_peaks()
     peak = float(peaks["bf16_tflops"])
-    achieved = flops / (ms_step * 1e-3) / 1e12
+    achieved = flops_rank / (ms_step * 1e-3) / 1e12
     traffic = None
     traffic_note = "no ncu capture of this kernel version"
     if os.path.exists(TRAFFIC_FILE):
@@ -313,11 +360,19 @@ def run_native(args, rank, world, local_rank):
         cpu = {"value": tf, "unit": UNIT, "cores": thr, "kind": "oracle",
                "sample": f"{nrows} random query rows of the same workload (fp64, all their visible keys), "
                          f"{secs:.1f} s"}
+    cfg = workload_config(w0, world)
+    cfg.update({
+        "global_batch": wg.B,
+        "parallelism": (f"heads{world}: contiguous balanced ranges of the B*H = {wg.B * wg.H} heads "
+                        f"(fa_fwd_heads in place), {'O/LSE all-gathered' if args.allgather and world > 1 else 'no collective on the data path'}"),
+        "head_ranges": [list(r) for r in ranges],
+    })
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong" if args.strong else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(w0, world),
+        "config": cfg,
         "pct_of_spec_peak": 100.0 * value / world / SPEC_PEAK_TFLOPS,
         "pct_of_measured_peak": 100.0 * value / world / peak,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
@@ -326,13 +381,13 @@ def run_native(args, rank, world, local_rank):
                                     if peak_kind == "measured" else "fallback 1590 TFLOP/s",
                      "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"]),
                      "frac_of_spec_2250": achieved / SPEC_PEAK_TFLOPS,
-                     "algorithmic_flops_per_launch": flops, "traffic_note": traffic_note},
+                     "algorithmic_flops_per_launch": flops_rank, "traffic_note": traffic_note},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
         "gpu_launches": args.steps,
         "clocks": clk,
-        "kernel": "fa::fa_fwd_kernel<128, true> via fa_fwd_ws (dynamic schedule; libfa_fwd.so)",
+        "kernel": "fa::fa_fwd_kernel<128, true> via fa_fwd_heads (dynamic schedule; libfa_fwd.so)",
         "gpu_launches_note": "one fa_fwd_kernel launch per step (plus the library's 4-byte cudaMemsetAsync of the work counter)",
     }
     return line
@@ -608,6 +663,10 @@ def main():
     ap.add_argument("--atomic", action="store_true", help="with --backward: the non-deterministic variant")
     ap.add_argument("--ring", action="store_true", help="time ring attention of one sequence over the ranks")
     ap.add_argument("--proj", action="store_true", help="time attention + output projection (fa_fwd_proj)")
+    ap.add_argument("--strong", action="store_true",
+                    help="split the workload itself across the ranks (default: weak scaling, one workload per rank)")
+    ap.add_argument("--allgather", action="store_true",
+                    help="after the pass, all-gather every rank's O/LSE rows so each rank holds the whole result")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -33,6 +33,13 @@ class Workload:
     qk_std: float = 1.0
     v_std: float = 1.0
     seed: int = 42
+    # Structured inputs (both empty for the plain recipe).  If q_lead is given,
+    # element 0 of query row i of every (batch, head) is set to
+    # q_lead[i % len(q_lead)]; if k_lead is given, element 0 of key j is set to
+    # k_lead[(j // 128) % len(k_lead)] (one value per block of 128 keys).  The
+    # values replace the drawn ones before the rounding to the dtype.
+    q_lead: tuple = ()
+    k_lead: tuple = ()
 
     def q_shape(self):
         return (self.B, self.Sq, self.H, self.D) if self.layout == "BSND" else (self.B, self.H, self.Sq, self.D)
@@ -75,9 +82,23 @@ def make_qkv(w: Workload, device="cpu"):
     g = torch.Generator(device="cpu")
     g.manual_seed(int(w.seed))
     dt = DTYPES[w.dtype]
-    q = (torch.randn(w.q_shape(), generator=g, dtype=torch.float32) * w.qk_std).to(dt)
-    k = (torch.randn(w.kv_shape(), generator=g, dtype=torch.float32) * w.qk_std).to(dt)
+    q = torch.randn(w.q_shape(), generator=g, dtype=torch.float32) * w.qk_std
+    k = torch.randn(w.kv_shape(), generator=g, dtype=torch.float32) * w.qk_std
     v = (torch.randn(w.kv_shape(), generator=g, dtype=torch.float32) * w.v_std).to(dt)
+    seq_dim = 1 if w.layout == "BSND" else 2
+    if w.q_lead:
+        lead = torch.tensor(w.q_lead, dtype=torch.float32)
+        vals = lead[torch.arange(w.Sq) % len(w.q_lead)]
+        shape = [1, 1, 1]
+        shape[seq_dim] = w.Sq
+        q[..., 0] = vals.reshape(shape)
+    if w.k_lead:
+        lead = torch.tensor(w.k_lead, dtype=torch.float32)
+        vals = lead[(torch.arange(w.Sk) // 128) % len(w.k_lead)]
+        shape = [1, 1, 1]
+        shape[seq_dim] = w.Sk
+        k[..., 0] = vals.reshape(shape)
+    q, k = q.to(dt), k.to(dt)
     if device != "cpu":
         q, k, v = q.to(device), k.to(device), v.to(device)
     return q, k, v

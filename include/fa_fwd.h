@@ -150,6 +150,36 @@ fa_status fa_fwd_ws(const void *q, const void *k, const void *v, void *o, float 
 size_t fa_fwd_workspace_size(void);
 
 /*
+ * fa_fwd_heads -- the forward pass over a contiguous range of heads only:
+ * the share of one GPU when the heads of one problem are split across GPUs
+ * (page "64K long-sequence FlashAttention" (ai6s.net/6a140d07), section
+ * "performance tuning tips", multi-card model parallelism; attention heads
+ * are independent, so the split needs no exchange during the pass).
+ *
+ * q, k, v, o, lse, B .. dtype   as for fa_fwd: the WHOLE problem's tensors,
+ *                  in place.  Only the heads g = b * H + h (flattened, batch
+ *                  major) with head_begin <= g < head_begin + head_count are
+ *                  read and computed; their rows of o and lse are written and
+ *                  every other element of o and lse is left untouched.  So
+ *                  several calls over disjoint ranges (on one GPU, or on
+ *                  GPUs that each hold the tensors) together write the whole
+ *                  result, bit-identical to one fa_fwd call: a head's result
+ *                  does not depend on which launch computes it.
+ * head_begin, head_count   0 <= head_begin, head_begin + head_count <= B * H
+ *                  (else FA_ERR_INVALID_ARG); head_count = 0 is a no-op.
+ * workspace, workspace_bytes   as for fa_fwd_ws (dynamic schedule), or NULL
+ *                  and 0 for the static schedule of fa_fwd.
+ *
+ * Errors as for fa_fwd and fa_fwd_ws.  Asynchronous on `stream`; allocates
+ * nothing.
+ */
+fa_status fa_fwd_heads(const void *q, const void *k, const void *v, void *o, float *lse,
+                       int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D,
+                       fa_layout layout, int causal, float scale, fa_dtype dtype,
+                       int64_t head_begin, int64_t head_count,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * fa_fwd_varlen -- the same forward pass over a batch of B sequences of
  * different lengths, packed row after row (the uneven-work case of page "64K
  * long-sequence FlashAttention" (ai6s.net/6a140d07), section "multi-AI-Core

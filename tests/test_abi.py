@@ -194,6 +194,29 @@ def test_noalloc_reaches_device_checks(lib):
     assert call_noalloc(B=1 << 30, Sq=0) == fa.FA_ERR_UNSUPPORTED
 
 
+def call_heads(begin=0, count=2, ws=None, ws_bytes=0, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_fwd_heads(a.get("q", Q), a.get("k", K), a.get("v", V), a.get("o", O), a.get("lse", L),
+                           a["B"], a["H"], a["Sq"], a["Sk"], a["D"], a["layout"], a["causal"], a["scale"],
+                           a["dtype"], begin, count, ws, ws_bytes, None)
+
+
+def test_head_range_validation(lib):
+    """fa_fwd_heads: the range must lie in [0, B * H]; other arguments are checked as fa_fwd checks them."""
+    for begin, count in ((-1, 1), (0, -1), (0, 3), (2, 1), (3, 0)):
+        assert call_heads(begin, count) == fa.FA_ERR_INVALID_ARG, (begin, count)
+    for kw in (dict(B=0), dict(layout=3), dict(dtype=5), dict(scale=float("nan")), dict(D=96), dict(Sq=0),
+               dict(q=0), dict(o=O + 8), dict(o=Q)):
+        assert call_heads(**kw) == call(**kw), kw
+    assert call_heads(ws=WS, ws_bytes=4) == fa.FA_ERR_INVALID_ARG
+    assert call_heads(ws=WS + 4, ws_bytes=16) == fa.FA_ERR_MISALIGNED
+    assert call_heads(ws=Q + 64, ws_bytes=16) == fa.FA_ERR_ALIAS
+    # an empty range is a no-op; a valid call gets past the host checks (it fails later without a GPU)
+    assert call_heads(1, 0) == fa.FA_OK
+    assert call_heads(1, 1) not in (fa.FA_OK, fa.FA_ERR_INVALID_ARG, fa.FA_ERR_MISALIGNED, fa.FA_ERR_ALIAS)
+
+
 def call_selftest(limit_us=20000, **kw):
     a = dict(GOOD)
     a.update(kw)

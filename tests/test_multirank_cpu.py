@@ -1,8 +1,10 @@
 """Host logic of the multi-GPU benchmark path, run as two gloo ranks on the CPU.
 
-The forward pass shards by independent (batch, head) problems: every rank runs
-its own full workload and the only collectives are a barrier and a max of the
-timing.  These tests check that logic without a GPU.
+The forward pass shards by independent (batch, head) problems: under weak
+scaling each rank owns one workload's worth of heads, drawn from its own seed
+(rank_workload), and the only collectives are a barrier and a max of the
+timing.  These tests check that logic without a GPU; the partition itself and
+the reassembly of O are tested in test_shard_cpu.py.
 """
 import argparse
 import os
