@@ -39,12 +39,20 @@ FA_MERGE_FINAL = 2
 LAYOUTS = {"BSND": FA_BSND, "BHSD": FA_BHSD}
 
 # Names every public symbol of include/fa_fwd.h.
-EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_heads", "fa_fwd_noalloc", "fa_fwd_varlen",
+EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_opts", "fa_fwd_default_options",
+                    "fa_fwd_heads", "fa_fwd_noalloc", "fa_fwd_varlen",
                     "fa_bwd",
                     "fa_bwd_workspace_size", "fa_bwd_atomic",
                     "fa_bwd_atomic_workspace_size", "fa_lse_merge", "fa_out_proj", "fa_fwd_proj",
                     "fa_selftest_wait_timeout", "fa_device_status", "fa_query_support", "fa_status_string",
                     "fa_last_cuda_error", "fa_version")
+
+
+class FwdOptions(ctypes.Structure):
+    """The C fa_fwd_options: the lazy rescale's threshold and bf16 headroom (log2 units) and an
+    optional device pointer to four 64-bit branch counters."""
+    _fields_ = [("rescale_threshold_log2", ctypes.c_float), ("bf16_headroom_log2", ctypes.c_float),
+                ("branch_counts", ctypes.c_void_p)]
 
 
 class FaError(RuntimeError):
@@ -84,6 +92,11 @@ def load_library(path=None, rebuild_if_stale=True):
     lib.fa_fwd_ws.restype = c_int
     lib.fa_fwd_ws.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, vp,
                               ctypes.c_size_t, vp]
+    lib.fa_fwd_opts.restype = c_int
+    lib.fa_fwd_opts.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int,
+                                ctypes.POINTER(FwdOptions), vp, ctypes.c_size_t, vp]
+    lib.fa_fwd_default_options.restype = None
+    lib.fa_fwd_default_options.argtypes = [ctypes.POINTER(FwdOptions)]
     lib.fa_fwd_heads.restype = c_int
     lib.fa_fwd_heads.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, i64, i64,
                                  vp, ctypes.c_size_t, vp]
@@ -143,6 +156,22 @@ def fa_fwd_ws(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, wo
     lib = load_library()
     return lib.fa_fwd_ws(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
                          int(bool(causal)), float(scale), int(dtype), workspace, int(workspace_bytes), stream)
+
+
+def fa_fwd_default_options():
+    """The C fa_fwd_default_options: a FwdOptions holding the defaults fa_fwd uses."""
+    opts = FwdOptions()
+    load_library().fa_fwd_default_options(ctypes.byref(opts))
+    return opts
+
+
+def fa_fwd_opts(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, opts, workspace, workspace_bytes,
+                stream):
+    """The C fa_fwd_opts (opts: a FwdOptions or None) with raw pointers; returns the fa_status code."""
+    lib = load_library()
+    return lib.fa_fwd_opts(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout),
+                           int(bool(causal)), float(scale), int(dtype), ctypes.byref(opts) if opts is not None else None,
+                           workspace, int(workspace_bytes), stream)
 
 
 def fa_fwd_heads(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, head_begin, head_count,
@@ -281,7 +310,8 @@ def _dims(q, k, layout, head_num=None):
 
 
 def flash_attention_forward(q, k, v, layout="BSND", causal=False, scale=None, head_num=None,
-                            out=None, lse=None, stream=None, schedule="dynamic", workspace=None, heads=None):
+                            out=None, lse=None, stream=None, schedule="dynamic", workspace=None, heads=None,
+                            softmax_options=None):
     """Attention forward on CUDA tensors through the C ABI.
 
     q: [B, Sq, H, D] (BSND) or [B, H, Sq, D] (BHSD); k, v likewise with Sk.
@@ -294,6 +324,9 @@ def flash_attention_forward(q, k, v, layout="BSND", causal=False, scale=None, he
     heads=(head_begin, head_count) calls fa_fwd_heads instead: only the
     flattened heads b * H + h in that range are computed, in place in the
     whole tensors; the other heads' rows of out and lse are left as they were.
+    softmax_options (a dict with any of rescale_threshold_log2,
+    bf16_headroom_log2, branch_counts -- a CUDA int64 tensor of 4 counters the
+    kernel increments) calls fa_fwd_opts with those lazy-rescale settings.
     """
     import torch
     lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
@@ -319,6 +352,32 @@ def flash_attention_forward(q, k, v, layout="BSND", causal=False, scale=None, he
     if stream is None:
         stream = torch.cuda.current_stream(q.device) if q.is_cuda else None
     sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    if softmax_options is not None:
+        if heads is not None:
+            raise ValueError("softmax_options and heads cannot be combined")
+        opts = fa_fwd_default_options()
+        for key, val in softmax_options.items():
+            if key == "branch_counts":
+                if val.dtype != torch.int64 or val.numel() < 4 or not val.is_contiguous():
+                    raise ValueError("branch_counts must be a contiguous int64 tensor of 4 counters")
+                opts.branch_counts = val.data_ptr()
+            elif key in ("rescale_threshold_log2", "bf16_headroom_log2"):
+                setattr(opts, key, float(val))
+            else:
+                raise ValueError(f"unknown softmax option {key!r}")
+        wptr, wbytes = None, 0
+        if schedule == "dynamic":
+            nbytes = fa_fwd_workspace_size()
+            if workspace is None:
+                workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+            wptr, wbytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+        elif schedule != "static":
+            raise ValueError(f"schedule must be 'dynamic' or 'static', not {schedule!r}")
+        st = fa_fwd_opts(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                         B, H, Sq, Sk, D, lay, causal, scale, dt, opts, wptr, wbytes, sptr)
+        if st != FA_OK:
+            raise FaError(st, "fa_fwd_opts")
+        return out, lse
     if heads is not None:
         h0, hc = (int(x) for x in heads)
         wptr, wbytes = None, 0

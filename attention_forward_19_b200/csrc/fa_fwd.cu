@@ -73,21 +73,11 @@ constexpr int TMEM_COLS = 512;
 constexpr int BOX_BYTES = BM * 128;  // one 128-row x 64-element (128-byte) TMA box
 constexpr int UQ_DEPTH = 4;           // unit ids in flight between the producer and the consumers
 constexpr int UQ_CONSUMERS = 9;       // arrivals that free a unit-id slot: the MMA warp + 8 softmax warps
-#ifndef FA_RESCALE_LOG2
-#define FA_RESCALE_LOG2 15.0f
-#endif
-constexpr float RESCALE_LOG2 = FA_RESCALE_LOG2;  // O / l are rescaled only when a row max grows by more (log2 units)
-constexpr float RESCALE_POW2 = (float)(1u << (int)FA_RESCALE_LOG2);  // 2^RESCALE_LOG2
-#ifndef FA_HEADROOM_LOG2
-#define FA_HEADROOM_LOG2 8.0f
-#endif
-constexpr float HEADROOM_LOG2 = FA_HEADROOM_LOG2;  // bf16 only: a moved reference sits this far above the tile max
-// Test builds only (FA_COUNT_BRANCHES=1): per-warp counts of the softmax's
-// rarely taken branches, read back by fa_debug_branch_counts.  The product
-// build has neither the counters nor the entry point.
-#ifndef FA_COUNT_BRANCHES
-#define FA_COUNT_BRANCHES 0
-#endif
+// Defaults of the lazy rescale (fa_fwd_options): O / l are rescaled only when
+// a row max grows by more than the threshold (log2 units), and for bf16 a
+// moved reference sits the headroom above the tile max.
+constexpr float RESCALE_LOG2_DEFAULT = 15.0f;
+constexpr float HEADROOM_LOG2_DEFAULT = 8.0f;
 #ifndef FA_EMU_PAIRS
 #define FA_EMU_PAIRS 0
 #endif
@@ -148,18 +138,22 @@ struct Params {
   int total_q, total_k;
   uint8_t* o;           // O base (variable-length batch: rows of a ragged last tile are stored directly)
   long long lse_bs, lse_hs;   // LSE offsets of a batch and of a head (plus the packed row)
+  // Lazy rescale: the reference max moves only when a tile's max exceeds it
+  // by more than rescale_log2 (weights against a stale reference stay below
+  // rescale_pow2 = 2^rescale_log2); bf16 sets a moved reference headroom_log2
+  // above the tile max.
+  float rescale_log2, rescale_pow2, headroom_log2;
+  // Optional statistics (nullptr: off), per warp and key tile after a unit's
+  // first: [0] such warp-tiles, [1] speculative pass rejected (exact
+  // recompute), [2] O rescaled, [3] accepted with a weight above half the
+  // bound (a stale reference close to its limit).
+  unsigned long long* counts;
 };
 
 // Device error word: bit 0 a wait ran out (FA_ERR_TIMEOUT), bit 1 invalid
 // sequence offsets of a variable-length batch (FA_ERR_INVALID_ARG).
 __device__ int g_dev_error = 0;
 
-#if FA_COUNT_BRANCHES
-// [0] warp-tiles after a unit's first tile, [1] of them with the speculative
-// pass rejected (exact recompute), [2] with O rescaled, [3] accepted with a
-// weight above 2^(RESCALE_LOG2 - 1) (a stale reference close to its bound).
-__device__ unsigned long long g_branch_counts[4];
-#endif
 
 // ----------------------------------------------------------------------------- PTX helpers
 
@@ -898,6 +892,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tS = tmem + lane_bits + t * BM;
     const uint32_t tO = tmem + lane_bits + 2 * BM + t * D;
     const float c = p.scale_log2;
+    const float tau = p.rescale_log2, tau_pow2 = p.rescale_pow2;
+    const float headroom = BF16 ? p.headroom_log2 : 0.f;
     uint32_t s_use = 0, o_use = 0, e_use = 0;
     bool ok = true;
     uint8_t* sQt = smem + C::SMEM_Q + t * C::TILE_BYTES;
@@ -949,8 +945,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // 64 columns of S_t) only once accepted.  From the second tile on, the
         // exponentials are taken against the current reference m straight
         // away: the reference must move only if this tile's max exceeds it by
-        // more than RESCALE_LOG2, which shows as a weight above
-        // 2^RESCALE_LOG2.  Then (rarely) the warp reloads S (still intact in
+        // more than tau, which shows as a weight above 2^tau.  Then (rarely)
+        // the warp reloads S (still intact in
         // TMEM), takes the exact tile max, moves m and recomputes P.  The first
         // tile of a unit starts from the exact max.
         float p_top = 0.f, rowsum = 0.f;
@@ -959,17 +955,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         bool exact = (j == 0);
         if (!exact) {
           rowsum = exp_pack_row<BF16, EMU_PAIRS>(sr, cc, -m_use, pk, p_top);
-          exact = __any_sync(0xffffffffu, !(p_top <= RESCALE_POW2));
+          exact = __any_sync(0xffffffffu, !(p_top <= tau_pow2));
           if (exact) load_s(sr);
         }
         if (exact) {
           const float m_blk = row_max_scaled(sr, cc);
           const float m_cand = fmaxf(m, m_blk);
-          grow = (m == -INFINITY) || (m_cand > m + RESCALE_LOG2) || !(p_top <= RESCALE_POW2);
+          grow = (m == -INFINITY) || (m_cand > m + tau) || !(p_top <= tau_pow2);
           // bf16 keeps the fp32 exponent range, so the new reference is set
-          // above the max (weights <= 2^-HEADROOM) and later tiles may grow by
-          // HEADROOM + RESCALE_LOG2 before the next move; fp16 keeps the max.
-          if (grow) m = m_cand + (BF16 ? HEADROOM_LOG2 : 0.f);
+          // above the max (weights <= 2^-headroom) and later tiles may grow by
+          // headroom + tau before the next move; fp16 keeps the max.
+          if (grow) m = m_cand + headroom;
           m_use = (m == -INFINITY) ? 0.f : m;
           rowsum = exp_pack_row<BF16, EMU_PAIRS>(sr, cc, -m_use, pk, p_top);
         }
@@ -984,18 +980,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float corr = round_to_input<BF16>(p_top) - p_top;
         l = l * alpha + rowsum;
         ln = ln * alpha + rowsum + corr;
-#if FA_COUNT_BRANCHES
-        if (j > 0) {
+        if (p.counts != nullptr && j > 0) {
           const bool any_grow = __any_sync(0xffffffffu, grow);
-          const bool near = __any_sync(0xffffffffu, !exact && p_top > 0.5f * RESCALE_POW2);
+          const bool near = __any_sync(0xffffffffu, !exact && p_top > 0.5f * tau_pow2);
           if (lane == 0) {
-            atomicAdd(&g_branch_counts[0], 1ull);
-            if (exact) atomicAdd(&g_branch_counts[1], 1ull);
-            if (any_grow) atomicAdd(&g_branch_counts[2], 1ull);
-            if (near) atomicAdd(&g_branch_counts[3], 1ull);
+            atomicAdd(&p.counts[0], 1ull);
+            if (exact) atomicAdd(&p.counts[1], 1ull);
+            if (any_grow) atomicAdd(&p.counts[2], 1ull);
+            if (near) atomicAdd(&p.counts[3], 1ull);
           }
         }
-#endif
         if (j > 0 && __any_sync(0xffffffffu, grow)) {
           uint32_t orow[D];
           tmem_ld_cols<D / 32>(tO, orow);
@@ -1272,6 +1266,20 @@ struct SelfTest {
   unsigned long long wait_limit_ns;
 };
 
+// The lazy rescale's settings and the optional branch statistics (fa_fwd_options).
+struct SoftmaxOpts {
+  float rescale_log2 = fa::RESCALE_LOG2_DEFAULT;
+  float headroom_log2 = fa::HEADROOM_LOG2_DEFAULT;
+  unsigned long long* counts = nullptr;
+};
+
+void set_softmax_params(fa::Params& prm, const SoftmaxOpts& so) {
+  prm.rescale_log2 = so.rescale_log2;
+  prm.rescale_pow2 = exp2f(so.rescale_log2);
+  prm.headroom_log2 = so.headroom_log2;
+  prm.counts = so.counts;
+}
+
 // Every check of a dense forward call's arguments that needs no device, in
 // the order fa_fwd applies them.  FA_OK with *noop set: the call has no query
 // rows and nothing to do (the pointers are then not looked at).
@@ -1312,7 +1320,7 @@ fa_status host_checks(const void* q, const void* k, const void* v, const void* o
 fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
                    int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
                    unsigned int* sched, void* stream, const SelfTest* selftest = nullptr, int64_t head_begin = 0,
-                   int64_t head_count = -1) {
+                   int64_t head_count = -1, const SoftmaxOpts& so = SoftmaxOpts()) {
   // ---- arguments that need no device
   bool noop = false;
   fa_status hst = host_checks(q, k, v, o, lse, B, H, Sq, Sk, D, layout, scale, dtype, &noop);
@@ -1324,8 +1332,8 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
 
   // ---- device checks
   int dev = 0, sms = 0;
-  const void* ptrs[6] = {q, k, v, o, lse, sched};
-  fa_status st = device_checks(ptrs, 6, &dev, &sms);
+  const void* ptrs[7] = {q, k, v, o, lse, sched, so.counts};
+  fa_status st = device_checks(ptrs, 7, &dev, &sms);
   if (st != FA_OK) return st;
 
   CUtensorMap mq, mk, mv, mo;
@@ -1358,6 +1366,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   prm.wait_limit_ns = 1000000000ull;  // one second; a normal wait lasts microseconds
   prm.withhold_loads = 0;
+  set_softmax_params(prm, so);
   if (selftest) {
     prm.wait_limit_ns = selftest->wait_limit_ns;
     prm.withhold_loads = 1;
@@ -1471,6 +1480,52 @@ fa_status fa_fwd_ws(const void* q, const void* k, const void* v, void* o, float*
 
 size_t fa_fwd_workspace_size(void) { return kWorkspaceBytes; }
 
+void fa_fwd_default_options(fa_fwd_options* opts) {
+  if (!opts) return;
+  opts->rescale_threshold_log2 = fa::RESCALE_LOG2_DEFAULT;
+  opts->bf16_headroom_log2 = fa::HEADROOM_LOG2_DEFAULT;
+  opts->branch_counts = nullptr;
+}
+
+fa_status fa_fwd_opts(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                      int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
+                      const fa_fwd_options* opts, void* workspace, size_t workspace_bytes, void* stream) {
+  SoftmaxOpts so;
+  if (opts) {
+    const float t = opts->rescale_threshold_log2, h = opts->bf16_headroom_log2;
+    // weights against a stale reference reach 2^t, which must stay finite in fp16
+    if (!(t >= 0.f && t <= 15.f) || !(h >= 0.f && h <= 16.f)) return FA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(opts->branch_counts) & 7u) return FA_ERR_MISALIGNED;
+    so.rescale_log2 = t;
+    so.headroom_log2 = h;
+    so.counts = opts->branch_counts;
+  }
+  unsigned int* sched = nullptr;
+  if (workspace) {
+    if (workspace_bytes < kWorkspaceBytes) return FA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return FA_ERR_MISALIGNED;
+    sched = static_cast<unsigned int*>(workspace);
+  }
+  if (B > 0 && H > 0 && D > 0 && Sq > 0 && Sk > 0) {
+    const size_t qbytes = (size_t)(B * H * Sq * D) * 2, kvbytes = (size_t)(B * H * Sk * D) * 2;
+    const size_t lbytes = (size_t)(B * H * Sq) * 4;
+    const void* extra[2] = {workspace, so.counts};
+    const size_t extra_bytes[2] = {workspace_bytes, 4 * sizeof(unsigned long long)};
+    for (int i = 0; i < 2; ++i) {
+      const void* x = extra[i];
+      const size_t n = extra_bytes[i];
+      if (x && ((q && overlaps(x, n, q, qbytes)) || (k && overlaps(x, n, k, kvbytes)) ||
+                (v && overlaps(x, n, v, kvbytes)) || (o && overlaps(x, n, o, qbytes)) ||
+                (lse && overlaps(x, n, lse, lbytes))))
+        return FA_ERR_ALIAS;
+    }
+    if (workspace && so.counts && overlaps(workspace, workspace_bytes, so.counts, extra_bytes[1]))
+      return FA_ERR_ALIAS;
+  }
+  return fwd_impl(q, k, v, o, lse, B, H, Sq, Sk, D, layout, causal, scale, dtype, sched, stream, nullptr, 0, -1,
+                  so);
+}
+
 fa_status fa_fwd_heads(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
                        int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, int causal, float scale, fa_dtype dtype,
                        int64_t head_begin, int64_t head_count, void* workspace, size_t workspace_bytes,
@@ -1573,6 +1628,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
   prm.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   prm.wait_limit_ns = 1000000000ull;
   prm.withhold_loads = 0;
+  set_softmax_params(prm, SoftmaxOpts());
   return launch_units(prm, mq, mk, mv, mo, D, dtype, static_cast<unsigned int*>(workspace), dev, sms, stream);
 }
 
@@ -1599,17 +1655,6 @@ fa_status fa_device_status(void* stream) {
   return FA_OK;
 }
 
-#if FA_COUNT_BRANCHES
-// Test builds only: copies the four branch counters of the current device
-// (see g_branch_counts) to out[0..3] and zeroes them.  Synchronises the device.
-int fa_debug_branch_counts(unsigned long long* out) {
-  cudaError_t e = cudaDeviceSynchronize();
-  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(out, fa::g_branch_counts, 4 * sizeof(unsigned long long));
-  const unsigned long long zero[4] = {0ull, 0ull, 0ull, 0ull};
-  if (e == cudaSuccess) e = cudaMemcpyToSymbol(fa::g_branch_counts, zero, sizeof(zero));
-  return (int)e;
-}
-#endif
 
 fa_status fa_query_support(int64_t D, fa_dtype dtype) {
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_UNSUPPORTED;

@@ -150,6 +150,56 @@ fa_status fa_fwd_ws(const void *q, const void *k, const void *v, void *o, float 
 size_t fa_fwd_workspace_size(void);
 
 /*
+ * fa_fwd_options -- settings of the online softmax's lazy rescale, and
+ * optional statistics of it (for fa_fwd_opts).
+ *
+ * The pages' recurrence moves a row's running max, and rescales its running
+ * sum and partial output, whenever a key tile holds a larger logit (page
+ * "FlashAttention: long-text inference without running out of memory"
+ * (ai6s.net/6a0d42d8), section "tiling + online normalisation").  The kernel
+ * moves its reference max only when a tile's max exceeds it by more than
+ * rescale_threshold_log2 (in log2 units of the scaled logits); until then the
+ * tile's weights are taken against the older, smaller reference and may reach
+ * 2^rescale_threshold_log2.  O, the sum and the LSE use the same reference, so
+ * the result is the same softmax; only the rounding differs.  For bf16 a moved
+ * reference is set bf16_headroom_log2 above the tile max (weights then start
+ * at most 2^-headroom, so later tiles may rise further before the next move);
+ * fp16 ignores the headroom.  Threshold 0 and headroom 0 is the pages'
+ * recurrence taken literally.
+ *
+ * rescale_threshold_log2  in [0, 15] (fp16 holds weights up to 2^15); default 15.
+ * bf16_headroom_log2      in [0, 16]; default 8.
+ * branch_counts           NULL, or device memory for four 64-bit counters,
+ *                         8-byte aligned, that the kernel INCREMENTS (zero them
+ *                         first): per warp of 32 rows and key tile after a
+ *                         work unit's first, [0] such warp-tiles, [1] with the
+ *                         tile's speculative pass rejected (a weight above
+ *                         2^threshold: the tile is recomputed against its
+ *                         exact max), [2] with the rows' O rescaled, [3]
+ *                         accepted with a weight above 2^(threshold - 1).
+ */
+typedef struct fa_fwd_options {
+    float rescale_threshold_log2;
+    float bf16_headroom_log2;
+    unsigned long long *branch_counts;
+} fa_fwd_options;
+
+/* Fills *opts with the defaults fa_fwd uses (threshold 15, headroom 8, no counters). */
+void fa_fwd_default_options(fa_fwd_options *opts);
+
+/*
+ * fa_fwd_opts -- fa_fwd (workspace NULL) or fa_fwd_ws (workspace given) with
+ * the lazy rescale's settings and statistics taken from *opts (NULL: the
+ * defaults).  FA_ERR_INVALID_ARG for settings outside their ranges,
+ * FA_ERR_MISALIGNED / FA_ERR_NOT_DEVICE_POINTER / FA_ERR_ALIAS for the
+ * counters as for a tensor; otherwise as fa_fwd / fa_fwd_ws.
+ */
+fa_status fa_fwd_opts(const void *q, const void *k, const void *v, void *o, float *lse,
+                      int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D,
+                      fa_layout layout, int causal, float scale, fa_dtype dtype,
+                      const fa_fwd_options *opts, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * fa_fwd_heads -- the forward pass over a contiguous range of heads only:
  * the share of one GPU when the heads of one problem are split across GPUs
  * (page "64K long-sequence FlashAttention" (ai6s.net/6a140d07), section

@@ -194,6 +194,42 @@ def test_noalloc_reaches_device_checks(lib):
     assert call_noalloc(B=1 << 30, Sq=0) == fa.FA_ERR_UNSUPPORTED
 
 
+def call_opts(opts=None, ws=None, ws_bytes=0, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return fa.fa_fwd_opts(a.get("q", Q), a.get("k", K), a.get("v", V), a.get("o", O), a.get("lse", L),
+                          a["B"], a["H"], a["Sq"], a["Sk"], a["D"], a["layout"], a["causal"], a["scale"],
+                          a["dtype"], opts, ws, ws_bytes, None)
+
+
+def test_default_softmax_options(lib):
+    o = fa.fa_fwd_default_options()
+    assert (o.rescale_threshold_log2, o.bf16_headroom_log2, o.branch_counts) == (15.0, 8.0, None)
+
+
+def test_softmax_options_validation(lib):
+    """fa_fwd_opts: the settings' ranges, the counters' alignment and overlap; other arguments as fa_fwd."""
+    def opts(t=15.0, h=8.0, counts=None):
+        o = fa.FwdOptions()
+        o.rescale_threshold_log2, o.bf16_headroom_log2, o.branch_counts = t, h, counts
+        return o
+    for bad in (opts(t=-1.0), opts(t=15.5), opts(t=float("nan")), opts(h=-0.5), opts(h=17.0),
+                opts(h=float("inf"))):
+        assert call_opts(bad) == fa.FA_ERR_INVALID_ARG
+    assert call_opts(opts(counts=0x61000004)) == fa.FA_ERR_MISALIGNED
+    assert call_opts(opts(counts=Q + 64)) == fa.FA_ERR_ALIAS
+    assert call_opts(opts(counts=L)) == fa.FA_ERR_ALIAS
+    assert call_opts(opts(), ws=WS, ws_bytes=4) == fa.FA_ERR_INVALID_ARG
+    assert call_opts(opts(), ws=WS + 4, ws_bytes=16) == fa.FA_ERR_MISALIGNED
+    assert call_opts(opts(counts=WS + 8), ws=WS, ws_bytes=16) == fa.FA_ERR_ALIAS
+    for kw in (dict(B=0), dict(layout=3), dict(dtype=5), dict(scale=float("nan")), dict(D=96), dict(Sq=0),
+               dict(q=0), dict(o=O + 8), dict(o=Q)):
+        assert call_opts(None, **kw) == call_opts(opts(t=0.0, h=0.0), **kw) == call(**kw), kw
+    # valid settings get past the host checks (the call fails later without a GPU)
+    assert call_opts(opts(t=0.0, h=0.0)) not in (fa.FA_OK, fa.FA_ERR_INVALID_ARG, fa.FA_ERR_MISALIGNED,
+                                                  fa.FA_ERR_ALIAS)
+
+
 def call_heads(begin=0, count=2, ws=None, ws_bytes=0, **kw):
     a = dict(GOOD)
     a.update(kw)

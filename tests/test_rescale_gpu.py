@@ -19,25 +19,22 @@ q_lead / k_lead) so that the logits of chosen rows jump from tile to tile:
   under the acceptance bound (weights close to 2^15, in fp16 too), just over
   it, and deep falls.
 
-Each case is compared element by element with the fp64 oracle, through the
-product library.  A test-only build with branch counters (FA_COUNT_BRANCHES)
-runs the same inputs: its output must be bit-identical to the product's,
-and its counters must show that the branches ran.  A second test-only build
-with tau = 0 and no headroom (the reference max moves at every new maximum,
-the recurrence of page "FlashAttention: long-text inference without running
-out of memory", section "tiling + online normalisation", taken literally) is
-checked against the oracle on the same inputs, on the small parity shapes
-and on sampled rows of the full-size workloads.
+Each case is compared element by element with the fp64 oracle.  The same
+call with the library's branch counters on (fa_fwd_opts, branch_counts) must
+give bit-identical output, and its counters must show that the branches ran.
+The same library with threshold 0 and headroom 0 (the reference max moves at
+every new maximum: the recurrence of page "FlashAttention: long-text
+inference without running out of memory", section "tiling + online
+normalisation", taken literally) is checked against the oracle on the same
+inputs, on the small parity shapes and on sampled rows of the full-size
+workloads.
 """
-import ctypes
 import math
-import os
 
 import pytest
 import torch
 
 import attention_forward_19_b200 as fa
-from attention_forward_19_b200 import build as fa_build
 from fa_inputs import WORKLOADS, Workload, make_qkv, sample_rows
 from test_parity_gpu import SMALL, compare_full, compare_rows
 
@@ -90,64 +87,27 @@ CASES.append(ramp_case("bf16", "BHSD", True, 64, 1000, 1000, seed=320))
 CASES.append(sawtooth_case("fp16", "BSND", False, 64, 300, 2100, seed=420))
 
 
-class Variant:
-    """A test-only build of the library (attention_forward_19_b200.build.TEST_VARIANTS), loaded
-    next to the product library; only fa_fwd and fa_device_status are called."""
-
-    _cache = {}
-
-    @classmethod
-    def get(cls, name):
-        if name not in cls._cache:
-            path = fa_build.variant_path(name)
-            if os.path.exists(fa_build.NVCC):
-                fa_build.build_variant(name)
-            lib = ctypes.CDLL(path)
-            i64, vp, c_int, c_float = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-            lib.fa_fwd.restype = c_int
-            lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, c_float, c_int, vp]
-            lib.fa_device_status.restype = c_int
-            lib.fa_device_status.argtypes = [vp]
-            if name == "count":
-                lib.fa_debug_branch_counts.restype = c_int
-                lib.fa_debug_branch_counts.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
-            cls._cache[name] = lib
-        return cls._cache[name]
+TAU0 = {"rescale_threshold_log2": 0.0, "bf16_headroom_log2": 0.0}
 
 
-def run_variant(lib, w, q, k, v):
-    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
-    o = torch.empty_like(qd)
-    lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device="cuda")
-    stream = torch.cuda.current_stream().cuda_stream
-    st = lib.fa_fwd(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.Sq,
-                    w.Sk, w.D, fa.LAYOUTS[w.layout], int(w.causal), w.scale,
-                    fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP16, stream)
-    assert st == fa.FA_OK
-    assert lib.fa_device_status(stream) == fa.FA_OK
+def run(w, q, k, v, **opts):
+    o, lse = fa.flash_attention_forward(q.cuda(), k.cuda(), v.cuda(), layout=w.layout, causal=w.causal,
+                                        scale=w.scale, softmax_options=opts or None)
+    fa.check_device_status()
     return o, lse
-
-
-def branch_counts(lib):
-    out = (ctypes.c_ulonglong * 4)()
-    assert lib.fa_debug_branch_counts(out) == 0
-    return [int(x) for x in out]
 
 
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
 def test_forced_branches_against_oracle(orc, w):
     _need_gpu()
     q, k, v = make_qkv(w)
-    o, lse = fa.flash_attention_forward(q.cuda(), k.cuda(), v.cuda(), layout=w.layout, causal=w.causal,
-                                        scale=w.scale)
-    fa.check_device_status()
+    o, lse = run(w, q, k, v)
     compare_full(orc, w, q, k, v, o, lse)
 
-    # the counting build: same bits, and the branches ran
-    lib = Variant.get("count")
-    branch_counts(lib)                                  # zero the counters
-    o2, l2 = run_variant(lib, w, q, k, v)
-    total, rejected, rescaled, near = branch_counts(lib)
+    # the same call with the branch counters on: same bits, and the branches ran
+    counts = torch.zeros(4, dtype=torch.int64, device="cuda")
+    o2, l2 = run(w, q, k, v, branch_counts=counts)
+    total, rejected, rescaled, near = counts.tolist()
     assert torch.equal(o, o2) and torch.equal(lse, l2)
     print(f"BRANCHES {w.name}: warp-tiles {total} rejected {rejected} rescaled {rescaled} near-bound {near}")
     assert total > 0
@@ -159,26 +119,26 @@ def test_forced_branches_against_oracle(orc, w):
 
 
 @pytest.mark.parametrize("w", CASES + SMALL, ids=lambda w: w.name)
-def test_tau0_build_against_oracle(orc, w):
+def test_tau0_against_oracle(orc, w):
     _need_gpu()
     q, k, v = make_qkv(w)
-    o, lse = run_variant(Variant.get("tau0"), w, q, k, v)
+    o, lse = run(w, q, k, v, **TAU0)
     compare_full(orc, w, q, k, v, o, lse)
 
 
 @pytest.mark.parametrize("name", [n for n in WORKLOADS if n != "fp16_bsnd_b1_h2_s512_d64"])
-def test_tau0_build_full_size_sampled_rows(orc, name):
+def test_tau0_full_size_sampled_rows(orc, name):
     _need_gpu()
     w = WORKLOADS[name]
     q, k, v = make_qkv(w)
-    o, lse = run_variant(Variant.get("tau0"), w, q, k, v)
+    o, lse = run(w, q, k, v, **TAU0)
     rows = sample_rows(w, per_head_first=16, per_head_last=16, stride=509, max_rows=3000)
     compare_rows(orc, w, q, k, v, o, lse, rows)
 
 
-def test_tau0_build_small_workload(orc):
+def test_tau0_small_workload(orc):
     _need_gpu()
     w = WORKLOADS["fp16_bsnd_b1_h2_s512_d64"]
     q, k, v = make_qkv(w)
-    o, lse = run_variant(Variant.get("tau0"), w, q, k, v)
+    o, lse = run(w, q, k, v, **TAU0)
     compare_full(orc, w, q, k, v, o, lse)
