@@ -321,6 +321,17 @@ __device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// One lane of a converged warp: the lane that issues a group of tcgen05.mma.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(e));
+  return e != 0;
+}
+
 __device__ __forceinline__ void tc_commit_elect(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -777,7 +788,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t q_use[NQ] = {0, 0}, p_use[NQ] = {0, 0}, o_use[NQ] = {0, 0};
     bool ok = true;
     // K-major SW128 descriptors of the Q tiles and of ring slot 0; a slot or a
-    // 16-element K step only moves the start address (16-byte units).
+    // 16-element K step only moves the start address (16-byte units).  Each
+    // group of products is issued by one elected lane (one election per group:
+    // an election per instruction measured 2.5 % slower on the whole kernel).
     const uint64_t dQ0 = sdesc(sQ, 16, 1024);
     const uint64_t dKV0 = sdesc(sKV, 16, 1024);
     const uint64_t dV0 = sdesc(sKV, BOX_BYTES, 1024);
@@ -786,18 +799,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t a = dQ0 + (uint64_t)(t * TILE16);
       const uint64_t b = dKV0 + (uint64_t)(kslot * TILE16);
       const uint32_t d = tmem + t * BM;
+      if (elect_one()) {
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
-        mma_ss_elect(d, a + off, b + off, IDESC_QK, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
+          mma_ss(d, a + off, b + off, IDESC_QK, kk > 0 ? 1u : 0u);
+        }
       }
+      __syncwarp();
     };
     auto pv = [&](int t, uint32_t vslot, bool acc0) {
       const uint64_t b = dV0 + (uint64_t)(vslot * TILE16);
       const uint32_t d = tmem + 2 * BM + t * D, a = tmem + t * BM;
+      if (elect_one()) {
 #pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk)
-        mma_ts_elect(d, a + kk * 8, b + (uint64_t)(kk * 128), IDESC_PV, (acc0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(d, a + kk * 8, b + (uint64_t)(kk * 128), IDESC_PV, (acc0 || kk > 0) ? 1u : 0u);
+      }
+      __syncwarp();
     };
     uint32_t uq_pos = 0;
     while (ok) {
