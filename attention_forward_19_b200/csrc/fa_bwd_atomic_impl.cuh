@@ -187,12 +187,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       constexpr uint32_t SUBT16 = SUBT >> 4;
       const uint32_t tST = tmem + COL_ST, tDPT = tmem + COL_DPT, tDV = tmem + COL_DV, tDK = tmem + COL_DK;
       auto kmajor_products = [&](uint32_t d_tmem, uint64_t a, uint64_t bsub) {   // 128 x 64 over K = D
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < DH / 16; ++kk) {
-          const uint32_t offa = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
-          const uint32_t offb = (uint32_t)((kk >> 2) * (SUB_BOX >> 4) + (kk & 3) * 2);
-          mma_ss_elect(d_tmem, a + offa, bsub + offb, IDESC_ST, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < DH / 16; ++kk) {
+            const uint32_t offa = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
+            const uint32_t offb = (uint32_t)((kk >> 2) * (SUB_BOX >> 4) + (kk & 3) * 2);
+            mma_ss(d_tmem, a + offa, bsub + offb, IDESC_ST, kk > 0 ? 1u : 0u);
+          }
         }
+        __syncwarp();
       };
       auto q_k = [&](uint32_t u) { return dStrK + (uint64_t)((u % NST) * 2 * SUBT16); };
       auto do_k = [&](uint32_t u) { return dStrK + (uint64_t)((u % NST) * 2 * SUBT16 + SUBT16); };
@@ -215,9 +218,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = wait_bar(bar(W_A), u & 1u, abort_flag, limit);        // P^T(u) written
         if (!ok) break;
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < SUB / 16; ++kk)   // dV += P^T dO_u
-          mma_ts_elect(tDV, tST + packed_col64(kk), do_mn + (uint64_t)(kk * 128), IDESC_ACC, (u > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < SUB / 16; ++kk)   // dV += P^T dO_u
+            mma_ts(tDV, tST + packed_col64(kk), do_mn + (uint64_t)(kk * 128), IDESC_ACC, (u > 0 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
         const bool more = u + 1 < (uint32_t)nu;
         if (more) {
           ok = wait_bar(bar(ST_FULL + (u + 1) % NST), ((u + 1) / NST) & 1u, abort_flag, limit);
@@ -229,9 +235,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = wait_bar(bar(W_B), u & 1u, abort_flag, limit);        // dS^T(u) written
         if (!ok) break;
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < SUB / 16; ++kk)   // dK += dS^T Q_u
-          mma_ts_elect(tDK, tDPT + packed_col64(kk), q_mn + (uint64_t)(kk * 128), IDESC_ACC, (u > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < SUB / 16; ++kk)   // dK += dS^T Q_u
+            mma_ts(tDK, tDPT + packed_col64(kk), q_mn + (uint64_t)(kk * 128), IDESC_ACC, (u > 0 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
         tc_commit_elect(bar(ST_EMPTY + st));
         if (more) {
           kmajor_products(tDPT, dVk, do_k(u + 1));
@@ -244,9 +253,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_after();
         }
         const uint32_t tDQ = tmem + COL_DQ + qb * SUB;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)    // dQ^T = K^T dS^T(u)
-          mma_ss_elect(tDQ, dKmn + (uint64_t)(kk * 128), dDst + (uint64_t)(kk * 128), IDESC_DQ, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < BM / 16; ++kk)    // dQ^T = K^T dS^T(u)
+            mma_ss(tDQ, dKmn + (uint64_t)(kk * 128), dDst + (uint64_t)(kk * 128), IDESC_DQ, kk > 0 ? 1u : 0u);
+        }
+        __syncwarp();
         tc_commit_elect(bar(DQ_FULL + qb));
       }
       if (ok) tc_commit_elect(bar(ACC_FULL));

@@ -240,19 +240,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t tST = tmem, tDPT = tmem + BM, tDV = tmem + 2 * BM, tDK = tmem + 2 * BM + D;
       auto st_products = [&](uint32_t n) {     // S^T(n) = K Q_n^T
         const uint64_t q_k = dStr + (uint64_t)((n % NSTAGE) * 2 * TILE16);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
-          mma_ss_elect(tST, dK0 + off, q_k + off, IDESC_ST, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
+            mma_ss(tST, dK0 + off, q_k + off, IDESC_ST, kk > 0 ? 1u : 0u);
+          }
         }
+        __syncwarp();
       };
       auto dpt_products = [&](uint32_t n) {    // dP^T(n) = V dO_n^T
         const uint64_t do_k = dStr + (uint64_t)((n % NSTAGE) * 2 * TILE16 + TILE16);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
-          mma_ss_elect(tDPT, dV0k + off, do_k + off, IDESC_ST, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
+            mma_ss(tDPT, dV0k + off, do_k + off, IDESC_ST, kk > 0 ? 1u : 0u);
+          }
         }
+        __syncwarp();
       };
       // Order of the tensor work: S^T(0), dP^T(0), then per step n
       //   dV(n), S^T(n+1), dK(n), dP^T(n+1)
@@ -275,9 +281,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = wait_bar(bar(C::W_A), n & 1u, abort_flag, limit);     // P^T(n) written
         if (!ok) break;
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)    // dV += P^T dO_n  (P^T: 8 packed columns per 16 queries)
-          mma_ts_elect(tDV, tST + packed_col(kk), do_mn + (uint64_t)(kk * 128), IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BM / 16; ++kk)    // dV += P^T dO_n  (P^T: 8 packed columns per 16 queries)
+            mma_ts(tDV, tST + packed_col(kk), do_mn + (uint64_t)(kk * 128), IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
         const bool more = n + 1 < (uint32_t)nq;
         if (more) {
           ok = wait_bar(bar(C::ST_FULL + (n + 1) % NSTAGE), ((n + 1) / NSTAGE) & 1u, abort_flag, limit);
@@ -289,9 +298,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = wait_bar(bar(C::W_B), n & 1u, abort_flag, limit);     // dS^T(n) written
         if (!ok) break;
         tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)    // dK += dS^T Q_n
-          mma_ts_elect(tDK, tDPT + packed_col(kk), q_mn + (uint64_t)(kk * 128), IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BM / 16; ++kk)    // dK += dS^T Q_n
+            mma_ts(tDK, tDPT + packed_col(kk), q_mn + (uint64_t)(kk * 128), IDESC_ACC, (n > 0 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
         tc_commit_elect(bar(C::ST_EMPTY + st));
         if (more) {
           dpt_products(n + 1);
@@ -530,16 +542,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint64_t k_k = dStr + (uint64_t)((j % NSTAGE) * 2 * TILE16);
       const uint64_t v_k = k_k + TILE16;
       const uint32_t tS = s_buf(j);
+      if (elect_one()) {
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {   // S = Q K_j^T
-        const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
-        mma_ss_elect(tS, dQd + off, k_k + off, IDESC_S, kk > 0 ? 1u : 0u);
-      }
+        for (int kk = 0; kk < D / 16; ++kk) {   // S = Q K_j^T
+          const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
+          mma_ss(tS, dQd + off, k_k + off, IDESC_S, kk > 0 ? 1u : 0u);
+        }
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {   // dP = dO V_j^T
-        const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
-        mma_ss_elect(tDP, dDOd + off, v_k + off, IDESC_S, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < D / 16; ++kk) {   // dP = dO V_j^T
+          const uint32_t off = (uint32_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
+          mma_ss(tDP, dDOd + off, v_k + off, IDESC_S, kk > 0 ? 1u : 0u);
+        }
       }
+      __syncwarp();
     };
     if (ok) ok = wait_bar(bar(C::ST_FULL), 0, abort_flag, limit);
     if (ok) {
@@ -563,9 +578,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after();
       const uint64_t k_mn = dStrMN + (uint64_t)(st * 2 * TILE16);
       const uint32_t tS = s_buf(j);
+      if (elect_one()) {
 #pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk)    // dQ += dS K_j
-        mma_ts_elect(tDQ, tS + packed_col(kk), k_mn + (uint64_t)(kk * 128), IDESC_ACC, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BN / 16; ++kk)    // dQ += dS K_j
+          mma_ts(tDQ, tS + packed_col(kk), k_mn + (uint64_t)(kk * 128), IDESC_ACC, (j > 0 || kk > 0) ? 1u : 0u);
+      }
+      __syncwarp();
       tc_commit_elect(bar(C::ST_EMPTY + st));
     }
     if (ok) tc_commit_elect(bar(C::ACC_FULL));

@@ -105,6 +105,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       bool ok = true;
       uint32_t issued = 0;
+      // The weight is read by every token tile (it should stay in L2); a
+      // token tile's O rows are read by the CTAs of its few feature tiles at
+      // about the same time and then never again.
+      const uint64_t pol_w = l2_policy_evict_last(), pol_o = l2_policy_evict_first();
       for (int t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
         int b, s0, n0;
         tile_coords(t, b, s0, n0);
@@ -115,10 +119,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t dst = sbase + st * STAGE_BYTES;
           mbar_arrive_expect_tx(bar(FULL + st), STAGE_BYTES);
           const int h = kb / dbox, d0 = (kb - h * dbox) * TK;
-          tma_load_4d(dst, &tmO, bar(FULL + st), d0, p.bhsd ? s0 : h, p.bhsd ? h : s0, b);
+          tma_load_4d_hint(dst, &tmO, bar(FULL + st), d0, p.bhsd ? s0 : h, p.bhsd ? h : s0, b, pol_o);
           const int s1 = s0 + 128;            // may lie past S: the box is zero-filled
-          tma_load_4d(dst + A_HALF, &tmO, bar(FULL + st), d0, p.bhsd ? s1 : h, p.bhsd ? h : s1, b);
-          tma_load_4d(dst + A_BYTES, &tmW, bar(FULL + st), kb * TK, n0, 0, 0);
+          tma_load_4d_hint(dst + A_HALF, &tmO, bar(FULL + st), d0, p.bhsd ? s1 : h, p.bhsd ? h : s1, b, pol_o);
+          tma_load_4d_hint(dst + A_BYTES, &tmW, bar(FULL + st), kb * TK, n0, 0, 0, pol_w);
         }
       }
       const uint32_t first = issued > (uint32_t)NSTAGE ? issued - NSTAGE : 0u;
@@ -143,12 +147,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t src = sbase + st * STAGE_BYTES;
         const uint64_t da0 = sdesc(src, 16, 1024), da1 = sdesc(src + A_HALF, 16, 1024);
         const uint64_t db = sdesc(src + A_BYTES, 16, 1024);
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < TK / 16; ++kk) {
-          const uint32_t acc_in = (kb > 0 || kk > 0) ? 1u : 0u;
-          mma_ss_elect(tmem, da0 + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), IDESC, acc_in);
-          mma_ss_elect(tmem + TN, da1 + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), IDESC, acc_in);
+          for (int kk = 0; kk < TK / 16; ++kk) {
+            const uint32_t acc_in = (kb > 0 || kk > 0) ? 1u : 0u;
+            mma_ss(tmem, da0 + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), IDESC, acc_in);
+            mma_ss(tmem + TN, da1 + (uint64_t)(kk * 2), db + (uint64_t)(kk * 2), IDESC, acc_in);
+          }
         }
+        __syncwarp();
         tc_commit_elect(bar(EMPTY + st));
       }
       if (!ok) break;

@@ -304,23 +304,58 @@ def run_native(args, rank, world, local_rank):
         if rank == 0:
             print(f"{wg.name}: {ms_step:.4f} ms/step, {value:.1f} TFLOP/s (no e2e, no baseline)", flush=True)
         return None
-    # end to end through the public API: this rank's input rows from pinned host memory -> device ->
-    # kernel -> this rank's result rows (with --allgather, the whole result) back to pinned host memory
+    # End to end through the public API: this rank's input rows from pinned host memory -> device ->
+    # kernel -> this rank's result rows (with --allgather, the whole result) back to pinned host memory.
+    # The rank's heads are split into chunks that pipeline over three streams: the host-to-device copy
+    # of chunk g + 1 and the device-to-host copy of chunk g - 1 run while the kernel computes chunk g
+    # (fa_fwd_heads on the chunk's heads).
     e2e_steps = max(3, min(args.steps, 10))
-    dev_in = [view for t in (q, k, v) for view in shard.head_rows(t, h0, hc, wg.layout, wg.H)]
-    host_in = [view.cpu().pin_memory() for view in dev_in]
+    nchunk = max(1, min(args.e2e_chunks, hc)) if not (args.allgather and world > 1) else 1
+    bounds = [h0 + (hc * c) // nchunk for c in range(nchunk + 1)]
+    chunks = [(bounds[c], bounds[c + 1] - bounds[c]) for c in range(nchunk)]
+    dev_in = [[view for t in (q, k, v) for view in shard.head_rows(t, b0, n0, wg.layout, wg.H)] for b0, n0 in chunks]
+    host_in = [[view.cpu().pin_memory() for view in views] for views in dev_in]
     if args.allgather and world > 1:
-        dev_out = [o, lse]
+        dev_out = [[o, lse]]
     else:
-        dev_out = [view for t in (o, lse) for view in shard.head_rows(t, h0, hc, wg.layout, wg.H)]
-    host_out = [torch.empty(view.shape, dtype=view.dtype, pin_memory=True) for view in dev_out]
+        dev_out = [[view for t in (o, lse) for view in shard.head_rows(t, b0, n0, wg.layout, wg.H)]
+                   for b0, n0 in chunks]
+    host_out = [[torch.empty(view.shape, dtype=view.dtype, pin_memory=True) for view in views] for views in dev_out]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
     def e2e_step():
-        for dst, src in zip(dev_in, host_in):
-            dst.copy_(src, non_blocking=True)
-        step()
-        for dst, src in zip(host_out, dev_out):
-            dst.copy_(src, non_blocking=True)
+        start = torch.cuda.Event()
+        start.record(stream)
+        s_in.wait_event(start)
+        ready = []
+        for c in range(nchunk):
+            with torch.cuda.stream(s_in):
+                for dst, src in zip(dev_in[c], host_in[c]):
+                    dst.copy_(src, non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(s_in)
+                ready.append(e)
+        done = []
+        for c, (b0, n0) in enumerate(chunks):
+            stream.wait_event(ready[c])
+            fa.flash_attention_forward(q, k, v, layout=wg.layout, causal=wg.causal, scale=wg.scale, out=o,
+                                       lse=lse, stream=stream, schedule="dynamic", workspace=ws, heads=(b0, n0))
+            e = torch.cuda.Event()
+            e.record(stream)
+            done.append(e)
+        if args.allgather and world > 1:
+            shard.all_gather_heads(o, lse, ranges, wg.layout)
+            e = torch.cuda.Event()
+            e.record(stream)
+            done = [e]
+        for c in range(len(dev_out)):
+            s_out.wait_event(done[c])
+            with torch.cuda.stream(s_out):
+                for dst, src in zip(host_out[c], dev_out[c]):
+                    dst.copy_(src, non_blocking=True)
+        fin = torch.cuda.Event()
+        fin.record(s_out)
+        stream.wait_event(fin)
 
     e2e_step()
     barrier()
@@ -336,8 +371,8 @@ def run_native(args, rank, world, local_rank):
     e2e_ms = max_over_ranks(a0.elapsed_time(a1), world, dev)
     fa.check_device_status(stream)
     e2e_value = flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
-    h2d = sum(t.numel() * t.element_size() for t in host_in)
-    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    h2d = sum(t.numel() * t.element_size() for views in host_in for t in views)
+    d2h = sum(t.numel() * t.element_size() for views in host_out for t in views)
 
     if rank != 0:
         return None
@@ -384,7 +419,8 @@ def run_native(args, rank, world, local_rank):
                      "algorithmic_flops_per_launch": flops_rank, "traffic_note": traffic_note},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
+                "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+                "pipeline": f"{nchunk} head chunks over three streams (copy in, fa_fwd_heads, copy out)"},
         "gpu_launches": args.steps,
         "clocks": clk,
         "kernel": "fa::fa_fwd_kernel<128, true> via fa_fwd_heads (dynamic schedule; libfa_fwd.so)",
@@ -665,6 +701,8 @@ def main():
     ap.add_argument("--proj", action="store_true", help="time attention + output projection (fa_fwd_proj)")
     ap.add_argument("--strong", action="store_true",
                     help="split the workload itself across the ranks (default: weak scaling, one workload per rank)")
+    ap.add_argument("--e2e-chunks", type=int, default=8,
+                    help="head chunks of the end-to-end pipeline (1: copy in, compute, copy out in sequence)")
     ap.add_argument("--allgather", action="store_true",
                     help="after the pass, all-gather every rank's O/LSE rows so each rank holds the whole result")
     args = ap.parse_args()
