@@ -1254,6 +1254,11 @@ fa_status launch_units(fa::Params& prm, const CUtensorMap& mq, const CUtensorMap
                        void* stream) {
   const int grid = (int)(prm.total_units < sms ? prm.total_units : sms);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // With no more units than CTAs every CTA takes exactly its first unit, and
+  // the work counter would only be read to find nothing left: the launch then
+  // runs the static schedule (the same units, the same results) and the
+  // counter is not zeroed, which saves a memset on small, latency-bound calls.
+  if (prm.total_units <= grid) sched = nullptr;
   prm.sched = sched;
   if (sched) {
     cudaError_t e = cudaMemsetAsync(sched, 0, sizeof(unsigned int), s);

@@ -40,8 +40,9 @@
  * before P.V (fp32 accumulation); O is rounded to the input dtype once, at
  * the end; LSE is fp32.
  *
- * Besides the forward pass (fa_fwd, fa_fwd_ws, fa_fwd_noalloc, fa_fwd_varlen)
- * the library exports its backward pass (fa_bwd, fa_bwd_atomic), the merge of
+ * Besides the forward pass (fa_fwd, fa_fwd_ws, fa_fwd_opts, fa_fwd_heads,
+ * fa_fwd_noalloc, fa_fwd_varlen) the library exports its backward pass
+ * (fa_bwd, fa_bwd_atomic), the merge of
  * partial results that ring attention over several GPUs is built from
  * (fa_lse_merge), and the attention output projection (fa_out_proj,
  * fa_fwd_proj).  Each is described at its declaration below.
@@ -133,7 +134,9 @@ fa_status fa_fwd(const void *q, const void *k, const void *v, void *o, float *ls
  *
  * workspace        device memory of at least fa_fwd_workspace_size() bytes,
  *                  16-byte aligned, owned by the caller; the library zeroes
- *                  it on `stream` before the launch and uses it as scratch.
+ *                  it on `stream` before the launch and uses it as scratch
+ *                  (a call with no more work units than the GPU has SMs
+ *                  needs no counter: it neither zeroes nor uses it).
  *                  It must not overlap any tensor argument, and two calls
  *                  that may run at the same time need separate workspaces.
  * workspace_bytes  its size in bytes.
@@ -325,8 +328,9 @@ fa_status fa_selftest_wait_timeout(const void *q, const void *k, const void *v, 
  * with the device current); make that first call before any stream capture.
  * Only a successful lookup is kept: a lookup that fails returns FA_ERR_CUDA
  * and is tried again by the next call.  After cudaDeviceReset the kept
- * address is checked, found stale and looked up again.  Every call zeroes
- * the counter on `stream` before its launch and then uses it, so calls that
+ * address is checked, found stale and looked up again.  Every call that
+ * needs the counter (see fa_fwd_ws) zeroes it on `stream` before its launch
+ * and then uses it, so calls that
  * overlap on the same GPU (for example on two streams) race on it: serialise
  * them, or use fa_fwd_ws with separate workspaces.  Each GPU has its own copy
  * of the array.  Arguments, results and errors as for fa_fwd, checked in the
