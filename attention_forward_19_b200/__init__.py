@@ -491,8 +491,8 @@ def flash_attention_backward(q, k, v, o, lse, dout, layout="BSND", causal=False,
     (dL/dO) like o.  Returns (dq, dk, dv) shaped like q, k, v.  `workspace`, a
     uint8 CUDA tensor of fa_bwd_workspace_size(B, H, Sq) bytes
     (fa_bwd_atomic_workspace_size(B, H, Sq, D) when deterministic=False), is
-    allocated here when not given.  deterministic=False calls fa_bwd_atomic
-    (D = 128): one kernel per key tile, dQ added up in fp32 in any order.
+    allocated here when not given.  deterministic=False calls fa_bwd_atomic:
+    one kernel per key tile, dQ added up in fp32 in any order.
     Runs on `stream` without synchronising.
     """
     import torch

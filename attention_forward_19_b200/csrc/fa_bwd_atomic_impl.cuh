@@ -10,7 +10,7 @@
 // same as fa_bwd's (P = 2^(S c - LSE2), dS = P (dP - D), dV = P^T dO,
 // dK = scale dS^T Q, dQ = scale dS K).
 //
-// One CTA per 128-key tile walks the visible queries in steps of 64 (D = 128):
+// One CTA per 128-key tile walks the visible queries in steps of 64 (D = 64 or 128):
 //   S^T = K Q_u^T, dP^T = V dO_u^T         (keys on the TMEM lanes, 64 columns each)
 //   dV += P^T dO_u, dK += dS^T Q_u         (A from TMEM, as in fa_bwd)
 //   dQ_u^T = K^T dS_u^T                    (both operands from shared memory:
@@ -25,6 +25,10 @@
 // proxy fence and one thread issuing.)  A last kernel scales the accumulator
 // and rounds it into dq.  The 64-query step keeps the TMEM budget at 512
 // columns; the stream of Q / dO sub-tiles has three stages.
+// D = 64: dQ^T = K^T dS^T is still an M = 128 product (the layout the other
+// products use): the K tile's region holds two 64-column boxes as at D = 128,
+// the second one zeroed, so K^T read MN-major has 128 rows of which the last
+// 64 are zero, and so are dQ^T's last 64 TMEM lanes, which are not added.
 
 namespace fa {
 namespace bwda {
@@ -33,12 +37,10 @@ using bwd::LOAD_WARP;
 using bwd::MMA_WARP;
 using bwd::THREADS;
 
-constexpr int DH = 128;          // head dim of this kernel
 constexpr int SUB = 64;          // queries per step
 constexpr int NST = 3;           // streamed stages (a Q and a dO sub-tile, two vectors)
 constexpr int SUB_BOX = SUB * 128;            // one 64-row x 64-element box: 8 KB
-constexpr int TILE = BM * DH * 2;             // the K or V tile: 32 KB
-constexpr int SUBT = SUB * DH * 2;            // a Q or dO sub-tile: 16 KB
+constexpr int KT_BYTES = BM * 128 * 2;        // the K tile's region: two 64-column boxes, 32 KB
 constexpr int IN_FULL = 0;
 constexpr int ST_FULL = 1;
 constexpr int ST_EMPTY = ST_FULL + NST;
@@ -51,15 +53,25 @@ constexpr int RD_C = W_B + 1;                 // two: a dQ^T buffer read (256)
 constexpr int ACC_FULL = RD_C + 2;
 constexpr int DRAIN = ACC_FULL + 1;
 constexpr int NBAR = DRAIN + 1;
-constexpr int SMEM_FIX = 0;                               // K tile, V tile
-constexpr int SMEM_STREAM = 2 * TILE;                     // per stage: Q_u, dO_u sub-tiles
-constexpr int SMEM_DST = SMEM_STREAM + NST * 2 * SUBT;    // dS^T: 128 keys x 64 queries, 16-bit, swizzled
-constexpr int SMEM_VEC = SMEM_DST + BM * SUB * 2;         // per stage: lse2[64], dsum[64]
-constexpr int SMEM_BAR = SMEM_VEC + NST * 2 * SUB * 4;
-constexpr int SMEM_MISC = SMEM_BAR + NBAR * 8;
-constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;
-static_assert(SMEM_DST % 1024 == 0, "the swizzled dS^T tile needs 1024-byte alignment");
-static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
+
+template <int DH>
+struct ACfg {
+  static constexpr int VT_BYTES = BM * DH * 2;                     // the V tile
+  static constexpr int SUBT = SUB * DH * 2;                        // a Q or dO sub-tile
+  static constexpr int SMEM_FIX = 0;                               // K tile's region, then the V tile
+  static constexpr int SMEM_V = KT_BYTES;
+  static constexpr int SMEM_STREAM = KT_BYTES + VT_BYTES;          // per stage: Q_u, dO_u sub-tiles
+  static constexpr int SMEM_DST = SMEM_STREAM + NST * 2 * SUBT;    // dS^T: 128 keys x 64 queries, 16-bit, swizzled
+  static constexpr int SMEM_VEC = SMEM_DST + BM * SUB * 2;         // per stage: lse2[64], dsum[64]
+  static constexpr int SMEM_BAR = SMEM_VEC + NST * 2 * SUB * 4;
+  static constexpr int SMEM_MISC = SMEM_BAR + NBAR * 8;
+  static constexpr int SMEM_USED = SMEM_MISC + 16 + 1024;
+  // at least 120 KB, so that one CTA holds an SM (and its whole TMEM)
+  static constexpr int SMEM_BYTES = SMEM_USED > 122880 ? SMEM_USED : 122880;
+  static_assert(SMEM_DST % 1024 == 0, "the swizzled dS^T tile needs 1024-byte alignment");
+  static_assert(SMEM_STREAM % 1024 == 0, "streamed sub-tiles need 1024-byte alignment");
+  static_assert(SMEM_BYTES <= 232448, "shared memory of one CTA");
+};
 
 constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_ST = 256, COL_DPT = 320, COL_DQ = 384;
 
@@ -82,7 +94,8 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 // a 64-query step: group g packs its 32 queries into columns [32 g, 32 g + 16).
 __device__ __forceinline__ uint32_t packed_col64(int kk) { return (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8); }
 
-// The two 64-row boxes of one Q / dO sub-tile (rows s0 .. s0 + 63 of head h, batch b).
+// The 64-row boxes of one Q / dO sub-tile (rows s0 .. s0 + 63 of head h, batch b), one per 64 columns.
+template <int DH>
 __device__ __forceinline__ void load_sub(uint32_t dst, const CUtensorMap* map, uint32_t bar, int bhsd, int s0, int h,
                                          int b) {
 #pragma unroll
@@ -90,20 +103,22 @@ __device__ __forceinline__ void load_sub(uint32_t dst, const CUtensorMap* map, u
     tma_load_4d(dst + bx * SUB_BOX, map, bar, bx * 64, bhsd ? s0 : h, bhsd ? h : s0, b);
 }
 
-template <bool BF16>
+template <int DH, bool BF16>
 __global__ void __launch_bounds__(THREADS, 1)
     dkdvq_kernel(const __grid_constant__ bwd::Params p, const __grid_constant__ CUtensorMap tmQ64,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmDO64) {
+  using A = ACfg<DH>;
+  constexpr int SUBT = A::SUBT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t sFix = smem_u32(smem + SMEM_FIX);
-  const uint32_t sStr = smem_u32(smem + SMEM_STREAM);
-  const uint32_t sDst = smem_u32(smem + SMEM_DST);
-  const float* sVec = reinterpret_cast<const float*>(smem + SMEM_VEC);
-  const uint32_t bars = smem_u32(smem + SMEM_BAR);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + SMEM_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SMEM_MISC + 4);
+  const uint32_t sFix = smem_u32(smem + A::SMEM_FIX);
+  const uint32_t sStr = smem_u32(smem + A::SMEM_STREAM);
+  const uint32_t sDst = smem_u32(smem + A::SMEM_DST);
+  const float* sVec = reinterpret_cast<const float*>(smem + A::SMEM_VEC);
+  const uint32_t bars = smem_u32(smem + A::SMEM_BAR);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + A::SMEM_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + A::SMEM_MISC + 4);
   auto bar = [&](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t limit = p.wait_limit_ns;
@@ -141,6 +156,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
     tmem_relinquish();
   }
+  if constexpr (DH == 64) {
+    // the K tile's second 64-column box: zero rows of K^T read MN-major
+    if (warp < LOAD_WARP) {
+      uint4* z = reinterpret_cast<uint4*>(smem + A::SMEM_FIX + BOX_BYTES);
+      for (int i = threadIdx.x; i < BOX_BYTES / 16; i += LOAD_WARP * 32) z[i] = make_uint4(0, 0, 0, 0);
+      fence_proxy_async_smem();
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -148,14 +171,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   constexpr uint32_t FMT = BF16 ? 1u : 0u;
   constexpr uint32_t IDESC_ST = idesc_ab(BM, SUB, FMT, 0, 0);    // 128 keys x 64 queries, both K-major
   constexpr uint32_t IDESC_ACC = idesc_ab(BM, DH, FMT, 0, 1);    // 128 keys x D, A in TMEM, B MN-major
-  constexpr uint32_t IDESC_DQ = idesc_ab(DH, SUB, FMT, 1, 1);    // D x 64 queries, A and B MN-major
+  constexpr uint32_t IDESC_DQ = idesc_ab(BM, SUB, FMT, 1, 1);    // 128 (D, zero-padded) x 64 queries, MN-major
 
   if (warp == LOAD_WARP) {
     if (lane == 0 && nu > 0) {
       bool ok = true;
-      mbar_arrive_expect_tx(bar(IN_FULL), 2 * TILE);
+      mbar_arrive_expect_tx(bar(IN_FULL), 2 * A::VT_BYTES);
       bwd::load_tile(sFix, &tmK, bar(IN_FULL), DH / 64, p.bhsd, k0, h, b);
-      bwd::load_tile(sFix + TILE, &tmV, bar(IN_FULL), DH / 64, p.bhsd, k0, h, b);
+      bwd::load_tile(sFix + A::SMEM_V, &tmV, bar(IN_FULL), DH / 64, p.bhsd, k0, h, b);
       uint32_t issued = 0;
       for (int u = 0; u < nu && ok; ++u, ++issued) {
         const uint32_t st = issued % NST;
@@ -164,8 +187,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_arrive_expect_tx(bar(ST_FULL + st), 2 * SUBT + 2 * SUB * 4);
         const uint32_t dst = sStr + st * 2 * SUBT;
         const int q0 = (u_begin + u) * SUB;
-        load_sub(dst, &tmQ64, bar(ST_FULL + st), p.bhsd, q0, h, b);
-        load_sub(dst + SUBT, &tmDO64, bar(ST_FULL + st), p.bhsd, q0, h, b);
+        load_sub<DH>(dst, &tmQ64, bar(ST_FULL + st), p.bhsd, q0, h, b);
+        load_sub<DH>(dst + SUBT, &tmDO64, bar(ST_FULL + st), p.bhsd, q0, h, b);
         const size_t vo = (size_t)bh * p.Sq_pad + (size_t)q0;
         const uint32_t vdst = smem_u32(sVec + st * 2 * SUB);
         bwd::bulk_load(vdst, p.lse2 + vo, SUB * 4, bar(ST_FULL + st));
@@ -179,7 +202,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == MMA_WARP) {
     if (nu > 0) {
       bool ok = wait_bar(bar(IN_FULL), 0, abort_flag, limit);
-      const uint64_t dKk = sdesc(sFix, 16, 1024), dVk = sdesc(sFix + TILE, 16, 1024);
+      const uint64_t dKk = sdesc(sFix, 16, 1024), dVk = sdesc(sFix + A::SMEM_V, 16, 1024);
       const uint64_t dKmn = sdesc(sFix, BOX_BYTES, 1024);         // K^T: the K tile read MN-major
       const uint64_t dStrK = sdesc(sStr, 16, 1024);               // a sub-tile, K-major
       const uint64_t dStrMN = sdesc(sStr, SUB_BOX, 1024);         // a sub-tile, MN-major
@@ -280,7 +303,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     float* dq_acc_bh = p.dq_acc + (size_t)bh * p.Sq_pad * DH;
     bool ok = true;
     // phase C of step v: thread rit adds column rit of dQ_v (its 32 queries) to the
-    // accumulator; a warp's add covers 128 contiguous bytes of one query row
+    // accumulator; a warp's add covers 128 contiguous bytes of one query row.  At
+    // D = 64 the TMEM lanes 64-127 (zero rows) are read but not added.
     auto phase_c = [&](uint32_t v) -> bool {
       if (!wait_bar(bar(DQ_FULL + (v & 1u)), (v >> 1) & 1u, abort_flag, limit)) return false;
       tc_fence_after();
@@ -290,9 +314,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       reg_fence(r);
       tc_fence_before();
       mbar_arrive(bar(RD_C + (v & 1u)));
-      float* dst = dq_acc_bh + ((size_t)(u_begin + (int)v) * SUB + grp * 32) * DH + rit;
+      if (rit < DH) {
+        float* dst = dq_acc_bh + ((size_t)(u_begin + (int)v) * SUB + grp * 32) * DH + rit;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) atomicAdd(dst + (size_t)j * DH, __uint_as_float(r[j]));
+        for (int j = 0; j < 32; ++j) atomicAdd(dst + (size_t)j * DH, __uint_as_float(r[j]));
+      }
       return true;
     };
     for (uint32_t u = 0; u < (uint32_t)nu && ok; ++u) {
@@ -357,7 +383,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       {
         // row rit of the 128 x 64 tile, 16-byte chunks 4 grp .. 4 grp + 3, 128-byte swizzle
-        uint8_t* row = smem + SMEM_DST + rit * 128;
+        uint8_t* row = smem + A::SMEM_DST + rit * 128;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int chunk = (grp * 4 + j) ^ (rit & 7);
@@ -418,8 +444,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-// dq = scale * accumulator, rounded to the input dtype: one warp per query row, four columns per lane.
-template <bool BF16>
+// dq = scale * accumulator, rounded to the input dtype: one warp per query row, D / 32 columns per lane.
+template <int DH, bool BF16>
 __global__ void __launch_bounds__(256) dq_convert_kernel(const __grid_constant__ bwd::Params p) {
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -428,10 +454,16 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const __grid_constant__
   const int bh = (int)(row / p.Sq);
   const int i = (int)(row - (long long)bh * p.Sq);
   const int b = bh / p.H, h = bh - b * p.H;
-  const float4 a = *reinterpret_cast<const float4*>(p.dq_acc + ((size_t)bh * p.Sq_pad + i) * DH + lane * 4);
-  uint8_t* dst = p.dq + (size_t)b * p.q_bs + (size_t)h * p.q_hs + (size_t)i * p.q_rs + lane * 8;
-  *reinterpret_cast<uint2*>(dst) = make_uint2(pack2<BF16>(a.x * p.scale, a.y * p.scale),
-                                              pack2<BF16>(a.z * p.scale, a.w * p.scale));
+  const float* src = p.dq_acc + ((size_t)bh * p.Sq_pad + i) * DH;
+  uint8_t* dst = p.dq + (size_t)b * p.q_bs + (size_t)h * p.q_hs + (size_t)i * p.q_rs;
+  if constexpr (DH == 128) {
+    const float4 a = *reinterpret_cast<const float4*>(src + lane * 4);
+    *reinterpret_cast<uint2*>(dst + lane * 8) = make_uint2(pack2<BF16>(a.x * p.scale, a.y * p.scale),
+                                                           pack2<BF16>(a.z * p.scale, a.w * p.scale));
+  } else {
+    const float2 a = *reinterpret_cast<const float2*>(src + lane * 2);
+    *reinterpret_cast<uint32_t*>(dst + lane * 4) = pack2<BF16>(a.x * p.scale, a.y * p.scale);
+  }
 }
 
 }  // namespace bwda
@@ -441,31 +473,33 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const __grid_constant__
 
 namespace {
 
-bool g_bwda_configured[kMaxDevices][2];
+bool g_bwda_configured[kMaxDevices][4];
 
-template <bool BF16>
+template <int DH, bool BF16>
 fa_status launch_bwd_atomic(fa::bwd::Params& prm, const CUtensorMap& mq64, const CUtensorMap& mk,
                             const CUtensorMap& mv, const CUtensorMap& mdo64, int dev, cudaStream_t s) {
-  auto kern = fa::bwda::dkdvq_kernel<BF16>;
+  auto kern = fa::bwda::dkdvq_kernel<DH, BF16>;
+  constexpr int smem = fa::bwda::ACfg<DH>::SMEM_BYTES;
+  const int slot = (DH == 128 ? 0 : 2) + (BF16 ? 1 : 0);
   {
     std::lock_guard<std::mutex> g(g_dev_mu);
-    if (!g_bwda_configured[dev][BF16 ? 1 : 0]) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::bwda::SMEM_BYTES);
+    if (!g_bwda_configured[dev][slot]) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return cuda_fail((int)e);
-      g_bwda_configured[dev][BF16 ? 1 : 0] = true;
+      g_bwda_configured[dev][slot] = true;
     }
   }
   const long long rows = (long long)prm.B * prm.H * prm.Sq_pad;
-  fa::bwd::prep_kernel<128, BF16><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(prm);
+  fa::bwd::prep_kernel<DH, BF16><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail((int)e);
-  e = cudaMemsetAsync(prm.dq_acc, 0, (size_t)rows * 128 * sizeof(float), s);
+  e = cudaMemsetAsync(prm.dq_acc, 0, (size_t)rows * DH * sizeof(float), s);
   if (e != cudaSuccess) return cuda_fail((int)e);
-  kern<<<(unsigned)(prm.B * prm.H * prm.tk), fa::bwd::THREADS, fa::bwda::SMEM_BYTES, s>>>(prm, mq64, mk, mv, mdo64);
+  kern<<<(unsigned)(prm.B * prm.H * prm.tk), fa::bwd::THREADS, smem, s>>>(prm, mq64, mk, mv, mdo64);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail((int)e);
   const long long qrows = (long long)prm.B * prm.H * prm.Sq;
-  fa::bwda::dq_convert_kernel<BF16><<<(unsigned)((qrows + 7) / 8), 256, 0, s>>>(prm);
+  fa::bwda::dq_convert_kernel<DH, BF16><<<(unsigned)((qrows + 7) / 8), 256, 0, s>>>(prm);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail((int)e);
   return FA_OK;

@@ -775,7 +775,6 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
       15u)
     return FA_ERR_MISALIGNED;
   if (reinterpret_cast<uintptr_t>(lse) & 3u) return FA_ERR_MISALIGNED;
-  if (atomic && D != 128) return FA_ERR_UNSUPPORTED;
   const size_t wbytes = atomic ? bwd_atomic_workspace_size(B, H, Sq, D) : fa_bwd_workspace_size(B, H, Sq);
   if (workspace_bytes < wbytes) return FA_ERR_INVALID_ARG;
   const void* outs[4] = {dq, dk, dv, workspace};
@@ -843,8 +842,11 @@ fa_status bwd_impl(const void* q, const void* k, const void* v, const void* o, c
     CUtensorMap mq64, mdo64;
     if ((st = make_map(&mq64, q, dtype, layout, B, H, Sq, D, fa::bwda::SUB)) != FA_OK) return st;
     if ((st = make_map(&mdo64, dout, dtype, layout, B, H, Sq, D, fa::bwda::SUB)) != FA_OK) return st;
-    return dtype == FA_BF16 ? launch_bwd_atomic<true>(prm, mq64, mk, mv, mdo64, dev, s)
-                            : launch_bwd_atomic<false>(prm, mq64, mk, mv, mdo64, dev, s);
+    if (D == 128)
+      return dtype == FA_BF16 ? launch_bwd_atomic<128, true>(prm, mq64, mk, mv, mdo64, dev, s)
+                              : launch_bwd_atomic<128, false>(prm, mq64, mk, mv, mdo64, dev, s);
+    return dtype == FA_BF16 ? launch_bwd_atomic<64, true>(prm, mq64, mk, mv, mdo64, dev, s)
+                            : launch_bwd_atomic<64, false>(prm, mq64, mk, mv, mdo64, dev, s);
   }
   if (D == 128)
     return dtype == FA_BF16 ? launch_bwd<128, true>(prm, mq, mk, mv, mdo, dev, s, 0)

@@ -406,7 +406,7 @@ def run_native(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "strong" if args.strong else "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": wg.dtype, "data": "synthetic",
         "config": cfg,
         "pct_of_spec_peak": 100.0 * value / world / SPEC_PEAK_TFLOPS,
         "pct_of_measured_peak": 100.0 * value / world / peak,

@@ -344,7 +344,7 @@ fa_status fa_fwd_noalloc(const void *q, const void *k, const void *v, void *o, f
  * fa_bwd_atomic -- the backward pass's non-deterministic variant (page "catlass
  * FlashAttention template tuning" (hwcomputing.csdn.net/6a0d4681), section on
  * the backward: the `deterministic` switch, atomic adds when off).  Same
- * arithmetic and arguments as fa_bwd, D = 128 only (else FA_ERR_UNSUPPORTED).
+ * arithmetic and arguments as fa_bwd, D = 64 or 128.
  * One kernel per 128-key tile computes dK, dV and that tile's share of dQ;
  * the shares are added into an fp32 accumulator in the workspace by atomic
  * adds in whatever order the tiles finish, so dq may differ between runs by

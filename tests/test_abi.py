@@ -409,5 +409,8 @@ def test_bwd_atomic_workspace_and_validation(lib):
         a.update(kw)
         return fa.fa_bwd_atomic(Q, K, V, O, DO_, L, DQ, DK, DV, 1, 2, 64, 64, a["D"], fa.FA_BSND, 1, 0.125,
                                 fa.FA_BF16, WSB, a["ws_bytes"], None)
-    assert call(D=64) == fa.FA_ERR_UNSUPPORTED
+    assert call(D=96) == fa.FA_ERR_UNSUPPORTED
     assert call(ws_bytes=fa.fa_bwd_workspace_size(1, 2, 64)) == fa.FA_ERR_INVALID_ARG   # too small for dQ
+    # D = 64: its own accumulator size; a D = 128 workspace is large enough, a deterministic one is not
+    assert fa.fa_bwd_atomic_workspace_size(1, 2, 64, 64) == 2 * 128 * (2 + 64) * 4
+    assert call(D=64, ws_bytes=fa.fa_bwd_workspace_size(1, 2, 64)) == fa.FA_ERR_INVALID_ARG
