@@ -43,7 +43,8 @@ EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_opts
                     "fa_fwd_heads", "fa_fwd_noalloc", "fa_fwd_varlen",
                     "fa_bwd",
                     "fa_bwd_workspace_size", "fa_bwd_atomic",
-                    "fa_bwd_atomic_workspace_size", "fa_lse_merge", "fa_out_proj", "fa_fwd_proj",
+                    "fa_bwd_atomic_workspace_size", "fa_lse_merge", "fa_fwd_ring_step", "fa_out_proj",
+                    "fa_fwd_proj",
                     "fa_selftest_wait_timeout", "fa_device_status", "fa_query_support", "fa_status_string",
                     "fa_last_cuda_error", "fa_version")
 
@@ -53,6 +54,14 @@ class FwdOptions(ctypes.Structure):
     optional device pointer to four 64-bit branch counters."""
     _fields_ = [("rescale_threshold_log2", ctypes.c_float), ("bf16_headroom_log2", ctypes.c_float),
                 ("branch_counts", ctypes.c_void_p)]
+
+
+class RingSegment(ctypes.Structure):
+    """The C fa_ring_segment: query rows [row0, row0 + rows) against keys [key0, key0 + keys); a causal
+    offset >= 0 makes key c visible from row r iff c <= r + offset (< 0: no mask); first / last say
+    whether the rows have an earlier result to merge with and whether this result is final."""
+    _fields_ = [("row0", ctypes.c_int64), ("key0", ctypes.c_int64), ("keys", ctypes.c_int64),
+                ("causal_offset", ctypes.c_int64), ("first", ctypes.c_int32), ("last", ctypes.c_int32)]
 
 
 class FaError(RuntimeError):
@@ -110,6 +119,9 @@ def load_library(path=None, rebuild_if_stale=True):
                            vp, ctypes.c_size_t, vp]
     lib.fa_lse_merge.restype = c_int
     lib.fa_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, c_int, c_int, c_int, vp]
+    lib.fa_fwd_ring_step.restype = c_int
+    lib.fa_fwd_ring_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.POINTER(RingSegment),
+                                     c_int, c_int, c_float, c_int, vp, ctypes.c_size_t, vp]
     lib.fa_out_proj.restype = c_int
     lib.fa_out_proj.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_int, vp]
     lib.fa_fwd_proj.restype = c_int
@@ -214,6 +226,17 @@ def fa_lse_merge(o_part, lse_part, o_acc, lse_acc, o_out, lse_out, B, H, S, D, l
     lib = load_library()
     return lib.fa_lse_merge(o_part, lse_part, o_acc, lse_acc, o_out, lse_out, int(B), int(H), int(S), int(D),
                             int(layout), int(dtype), int(flags), stream)
+
+
+def fa_fwd_ring_step(q, k, v, o, acc, lse, B, H, Sq, Sk, D, rows, segs, layout, scale, dtype, workspace,
+                     workspace_bytes, stream):
+    """The C fa_fwd_ring_step with raw pointers; segs is a sequence of (row0, key0, keys, causal_offset,
+    first, last) tuples.  Returns the fa_status code."""
+    lib = load_library()
+    arr = (RingSegment * max(1, len(segs)))(*[RingSegment(*[int(x) for x in g]) for g in segs])
+    return lib.fa_fwd_ring_step(q, k, v, o, acc, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(rows), arr,
+                                len(segs), int(layout), float(scale), int(dtype), workspace, int(workspace_bytes),
+                                stream)
 
 
 def fa_out_proj(o, w_o, y, B, H, S, D, E, layout, dtype, stream):
@@ -582,6 +605,40 @@ def lse_merge(o_part, lse_part, o_acc=None, lse_acc=None, out=None, lse_out=None
     if st != FA_OK:
         raise FaError(st, "fa_lse_merge")
     return (out, lse_out) if final else (o_acc, lse_acc)
+
+
+def ring_step(q, k, v, segments, rows, out, lse, acc=None, layout="BSND", scale=None, workspace=None, stream=None):
+    """One ring-attention step through fa_fwd_ring_step: every segment (row0, key0, keys, causal_offset,
+    first, last) attends its query rows of q to its keys of k / v and merges the result into the running
+    result of those rows (acc fp32 like q, lse fp32 [B, H, Sq]), or writes the final one to out / lse.
+
+    q, out: [B, Sq, H, D] (BSND) or [B, H, Sq, D] (BHSD); k, v likewise with Sk rows; all contiguous CUDA
+    tensors.  scale=None uses 1/sqrt(D).  Asynchronous on `stream` (default: the current torch stream)."""
+    import torch
+    lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    B, H, Sq, Sk, D = _dims(q, k, lay)
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if v.shape != k.shape or out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("v must be shaped like k and out like q")
+    if lse.shape != (B, H, Sq) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 tensor of shape [B, H, Sq]")
+    if acc is not None and (acc.shape != q.shape or acc.dtype != torch.float32 or not acc.is_contiguous()):
+        raise ValueError("acc must be a contiguous fp32 tensor shaped like q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if workspace is None:
+        workspace = torch.empty(fa_fwd_workspace_size(), dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    st = fa_fwd_ring_step(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                          acc.data_ptr() if acc is not None else None, lse.data_ptr(), B, H, Sq, Sk, D, rows,
+                          segments, lay, scale, _dtype_code(q), workspace.data_ptr(), workspace.numel(), sptr)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_ring_step")
+    return out, lse
 
 
 def _proj_dims(o, w_o, lay):

@@ -9,7 +9,8 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "fa_fwd.cu")
-DEPS = [os.path.join(PKG, "csrc", n) for n in ("fa_bwd_impl.cuh", "fa_merge_impl.cuh", "fa_proj_impl.cuh")]   # included by fa_fwd.cu
+DEPS = [os.path.join(PKG, "csrc", n) for n in ("fa_bwd_impl.cuh", "fa_bwd_atomic_impl.cuh", "fa_merge_impl.cuh",
+                                            "fa_proj_impl.cuh")]   # included by fa_fwd.cu
 HDR = os.path.join(ROOT, "include", "fa_fwd.h")
 LIB = os.path.join(PKG, "libfa_fwd.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -136,8 +136,20 @@ struct Params {
   const int* cu_q;
   const int* cu_k;
   int total_q, total_k;
-  uint8_t* o;           // O base (variable-length batch: rows of a ragged last tile are stored directly)
-  long long lse_bs, lse_hs;   // LSE offsets of a batch and of a head (plus the packed row)
+  uint8_t* o;           // O base (packed and ring-step launches store each row directly)
+  long long o_bs, o_hs, o_rs;  // element offsets in O of a batch, a head and a row (row stores)
+  long long lse_bs, lse_hs;   // LSE offsets of a batch and of a head (plus the row)
+  // Ring step: nseg (1 or 2) query segments with disjoint rows, segment 0's
+  // units first (seg_units0 of them).  Segment s takes query rows
+  // [seg_row0[s], seg_row0[s] + Sq) of Q / O / LSE and keys
+  // [seg_key0[s], seg_key0[s] + seg_sk[s]) of K / V; with seg_causal[s], key c
+  // of the segment is visible from its row r iff c <= r + seg_coff[s].
+  // seg_flags[s]: bit 0 (first) no earlier result to merge, bit 1 (last) the
+  // merged result is final (O in the input dtype); otherwise it is the running
+  // result: fp32 O in acc (strides of O) and its LSE in lse.
+  int nseg, seg_units0;
+  int seg_row0[2], seg_key0[2], seg_sk[2], seg_coff[2], seg_causal[2], seg_flags[2];
+  float* acc;
   // Lazy rescale: the reference max moves only when a tile's max exceeds it
   // by more than rescale_log2 (weights against a stale reference stay below
   // rescale_pow2 = 2^rescale_log2); bf16 sets a moved reference headroom_log2
@@ -413,6 +425,10 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[32 * 
   reg_fence(r);
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -593,31 +609,48 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, uint32_t fmt, uin
 
 // ----------------------------------------------------------------------------- schedule
 
+// Launch kinds (the kernel's KIND): a dense batch, a packed variable-length
+// batch, a ring step (query segments merged into a running result).
+constexpr int DENSE = 0, PACKED = 1, RING = 2;
+
 struct Unit {
   int b, h, r0;     // batch, head, first query row of the unit (within its sequence)
+  int causal, coff; // causal mask (key c visible from row r iff c <= r + coff)
+  int seg;          // ring-step segment
   int rows[NQ];     // valid rows of each query tile
   int n[NQ];        // key tiles each query tile visits (0: tile inactive)
   int sq, sk;       // the sequence's query and key lengths
-  int rb, kb;       // its first packed query row and key row (0 for a dense batch)
+  int rb, kb;       // its first query row and key row in the tensors (0 for a dense batch)
   int tb;           // batch coordinate of the tensor maps (0 for a packed batch)
 };
 
 // Units are grouped by heads so that the K / V of a group stay in L2; inside
 // a group the longest units (causal: the last query rows) come first.
-template <bool VARLEN>
+template <int KIND>
 __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
+  Unit un;
+  un.causal = p.causal;
+  un.coff = 0;
+  un.seg = 0;
+  if constexpr (KIND == RING) {
+    // (selects rather than indexing: a dynamic index into the parameters
+    // would copy them to local memory)
+    un.seg = u >= p.seg_units0 ? 1 : 0;
+    if (un.seg) u -= p.seg_units0;
+    un.causal = un.seg ? p.seg_causal[1] : p.seg_causal[0];
+    un.coff = un.seg ? p.seg_coff[1] : p.seg_coff[0];
+  }
   const int per_group = p.group_heads * p.nqb;
   const int g = u / per_group;
   const int r = u - g * per_group;
   const int gs = min(p.group_heads, p.bh - g * p.group_heads);
   const int level = r / gs;
   const int bh = p.head0 + g * p.group_heads + (r - level * gs);
-  const int qblk = p.causal ? (p.nqb - 1 - level) : level;
-  Unit un;
+  const int qblk = un.causal ? (p.nqb - 1 - level) : level;
   un.b = bh / p.H;
   un.h = bh - un.b * p.H;
   un.r0 = qblk * UNIT_ROWS;
-  if constexpr (VARLEN) {
+  if constexpr (KIND == PACKED) {
     // Every role decodes the same offsets.  Offsets that cannot describe a
     // sequence of this batch (and a sequence with queries but no keys) make
     // the unit empty and are reported in the device error word.
@@ -630,6 +663,12 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
     un.rb = q0;
     un.kb = k0;
     un.tb = 0;
+  } else if constexpr (KIND == RING) {
+    un.sq = p.Sq;
+    un.sk = un.seg ? p.seg_sk[1] : p.seg_sk[0];
+    un.rb = un.seg ? p.seg_row0[1] : p.seg_row0[0];
+    un.kb = un.seg ? p.seg_key0[1] : p.seg_key0[0];
+    un.tb = un.b;
   } else {
     un.sq = p.Sq;
     un.sk = p.Sk;
@@ -644,8 +683,8 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
     un.rows[t] = rows;
     if (rows == 0) {
       un.n[t] = 0;
-    } else if (p.causal) {
-      const int last_key = min(first + rows - 1, un.sk - 1);
+    } else if (un.causal) {
+      const int last_key = min(first + rows - 1 + un.coff, un.sk - 1);
       un.n[t] = last_key / BN + 1;
     } else {
       un.n[t] = (un.sk + BN - 1) / BN;
@@ -656,12 +695,16 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
 
 // ----------------------------------------------------------------------------- kernel
 
-template <int D, bool BF16, bool VARLEN>
+template <int D, bool BF16, int KIND>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmO) {
   using C = Cfg<D>;
+  // Packed and ring-step launches store O row by row from registers (a tile
+  // may end inside a sequence or a segment, where a TMA store would also
+  // write the next one's rows), so Q is released after its last read.
+  constexpr bool ROWSTORE = KIND != DENSE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sQ = smem_u32(smem + C::SMEM_Q);
@@ -685,9 +728,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar(C::Q_FULL + t), 1);
       mbar_init(bar(C::Q_EMPTY + t), 1);
       mbar_init(bar(C::S_FULL + t), 1);
-      mbar_init(bar(C::P_FULL + t), BM);
+      mbar_init(bar(C::P_FULL + t), BM / 32);   // one arrival per softmax warp
       mbar_init(bar(C::O_FULL + t), 1);
-      mbar_init(bar(C::O_EMPTY + t), BM);
+      mbar_init(bar(C::O_EMPTY + t), BM / 32);
       mbar_init(bar(C::EPI + t), BM);
     }
     mbar_init(bar(C::DRAIN), 1);
@@ -740,7 +783,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           u += (int)gridDim.x;
           continue;
         }
-        const Unit un = decode_unit<VARLEN>(p, u);
+        const Unit un = decode_unit<KIND>(p, u);
         const int n = max(un.n[0], un.n[1]);
 #pragma unroll
         for (int t = 0; t < NQ; ++t) {
@@ -831,9 +874,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) mbar_arrive(bar(C::UQ_EMPTY + qs));
       ++uq_pos;
       if (u >= p.total_units) break;
-      const Unit un = decode_unit<VARLEN>(p, u);
+      const Unit un = decode_unit<KIND>(p, u);
       const int n = max(un.n[0], un.n[1]);
-      if (VARLEN && n == 0) continue;   // an empty sequence of a variable-length batch
+      if (KIND == PACKED && n == 0) continue;   // an empty sequence of a variable-length batch
 #pragma unroll
       for (int t = 0; t < NQ; ++t) {
         if (un.n[t] == 0 || !ok) continue;
@@ -854,7 +897,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_commit_elect(bar(C::S_FULL + t));
         // packed batch: Q_t is read by no later MMA, so the producer may load
         // the next unit's Q_t as soon as this one completes
-        if (VARLEN && un.n[t] == 1) tc_commit_elect(bar(C::Q_EMPTY + t));
+        if (ROWSTORE && un.n[t] == 1) tc_commit_elect(bar(C::Q_EMPTY + t));
       }
       tc_commit_elect(bar(C::KV_EMPTY + kslot));
       for (int j = 0; j < n && ok; ++j) {
@@ -891,7 +934,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // softmax may rescale O_t once it has seen S_t(j+1).
             qk(t, kslot);
             tc_commit_elect(bar(C::S_FULL + t));
-            if (VARLEN && j + 2 == un.n[t]) tc_commit_elect(bar(C::Q_EMPTY + t));   // last read of Q_t
+            if (ROWSTORE && j + 2 == un.n[t]) tc_commit_elect(bar(C::Q_EMPTY + t));   // last read of Q_t
           }
         }
         if (!ok) break;
@@ -930,7 +973,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) mbar_arrive(bar(C::UQ_EMPTY + qs));
       ++uq_pos;
       if (u >= p.total_units) break;
-      const Unit un = decode_unit<VARLEN>(p, u);
+      const Unit un = decode_unit<KIND>(p, u);
       const int nt = t ? un.n[1] : un.n[0];
       if (nt == 0) continue;
       const int row = un.r0 + t * BM + rit;          // query row of this thread
@@ -939,17 +982,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       float l = 0.f;                                 // running exp-sum (for the LSE)
       float ln = 0.f;                                // l with each tile's top weight as rounded in P (for O)
       float m_use = 0.f;
+      const int seg_flags = KIND == RING ? (un.seg ? p.seg_flags[1] : p.seg_flags[0]) : 0;
       for (int j = 0; j < nt; ++j) {
+        if constexpr (KIND == RING) {
+          // the running O row the epilogue merges with: into L2 while the last tile is computed
+          if (j + 1 == nt && !(seg_flags & 1) && row < un.sq) {
+            const float* a = p.acc + (size_t)un.b * p.o_bs + (size_t)un.h * p.o_hs + (size_t)(un.rb + row) * p.o_rs;
+#pragma unroll
+            for (int i = 0; i < D / 32; ++i) prefetch_l2(a + 32 * i);
+          }
+        }
         // S_t(j) is complete; its commit also covers P_t(j-1) V(j-1), so O_t is settled.
         ok = wait_bar(bar(C::S_FULL + t), s_use & 1u, abort_flag, limit);
         if (!ok) break;
         ++s_use;
         tc_fence_after();
         const int c0 = j * BN;
-        const bool masked = (c0 + BN > un.sk) || (p.causal && (c0 + BN - 1 > first_row));
+        const bool masked = (c0 + BN > un.sk) || (un.causal && (c0 + BN - 1 > first_row + un.coff));
         const float cc = masked ? 1.f : c;
         int lim = un.sk - 1 - c0;
-        if (p.causal) lim = min(lim, row - c0);
+        if (un.causal) lim = min(lim, row + un.coff - c0);
         // this row of S_t from TMEM; diagonal / ragged tiles become scaled logits
         // with masked entries at -inf
         auto load_s = [&](uint32_t (&sr)[BN]) {
@@ -1029,7 +1081,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(C::P_FULL + t));
+        // every lane's P (and rescaled O) stores are complete: one arrival per warp
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::P_FULL + t));
       }
       if (!ok) break;
 
@@ -1038,28 +1092,81 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       ++o_use;
       tc_fence_after();
-      const float inv_l = 1.f / ln;
       // Dense batch: O is staged (swizzled) in the Q tile's buffer and stored
       // by TMA; the buffer is released once the store has read it.  Packed
-      // (variable-length) batch: each thread stores its own row from
-      // registers -- a tile may end inside the sequence, where a TMA store
-      // would also write the next sequence's rows -- and the MMA warp has
-      // already released the Q buffer after its last read.
+      // batch and ring step: each thread stores its own row from registers,
+      // and the MMA warp has already released the Q buffer after its last read.
       const bool store_row = row < un.sq;
+      const size_t lse_at = (size_t)un.b * p.lse_bs + (size_t)un.h * p.lse_hs + un.rb + row;
+      float lse2 = m_use + lg2(l);          // this result's LSE (log2 units)
+      float w_o = 1.f / ln;                 // O = w_o * O_tmem (+ w_run * running O)
+      float w_run = 0.f;
+      bool merge = false, final_o = true;
       uint8_t* orow = nullptr;
-      if constexpr (VARLEN) orow = p.o + ((size_t)(un.rb + row) * p.H + un.h) * (D * 2);
+      float* arow = nullptr;
+      if constexpr (ROWSTORE) {
+        const size_t e = (size_t)un.b * p.o_bs + (size_t)un.h * p.o_hs + (size_t)(un.rb + row) * p.o_rs;
+        orow = p.o + e * 2;
+        if constexpr (KIND == RING) arow = p.acc + e;
+      }
+      if constexpr (KIND == RING) {
+        // Merge with the running result (LSE a): the merged LSE is
+        // log2(2^a + 2^lse2) and each part is weighted by 2^(its LSE - merged).
+        final_o = (seg_flags & 2) != 0;
+        merge = !(seg_flags & 1) && store_row;
+        if (merge) {
+          const float a = p.lse[lse_at] * 1.44269504088896340736f;
+          const float mx = fmaxf(a, lse2);
+          const float ea = ex2(a - mx), eb = ex2(lse2 - mx);
+          const float inv = 1.f / (ea + eb);
+          w_run = ea * inv;
+          w_o *= eb * inv;
+          lse2 = mx + lg2(ea + eb);
+        }
+      }
       {
         uint32_t r[32];
-#pragma unroll
+        float4 run[8];     // 32 columns of the running O row
+        // (a ring step keeps this loop rolled: unrolled, the running O loads
+        // of every chunk are hoisted together and the registers spill)
+#pragma unroll(KIND == RING ? 1 : D / 32)
         for (int q4 = 0; q4 < D / 32; ++q4) {
+          if constexpr (KIND == RING) {
+            if (merge) {
+              const float4* src = reinterpret_cast<const float4*>(arow) + q4 * 8;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) run[i] = src[i];
+            }
+          }
           tmem_ld32(tO + q4 * 32, r);
           tmem_wait_ld();
           reg_fence(r);
+          float f[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(r[i]) * w_o;
+          if constexpr (KIND == RING) {
+            if (merge) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                f[4 * i] += run[i].x * w_run;
+                f[4 * i + 1] += run[i].y * w_run;
+                f[4 * i + 2] += run[i].z * w_run;
+                f[4 * i + 3] += run[i].w * w_run;
+              }
+            }
+            if (!final_o) {
+              if (store_row) {
+                float4* dst = reinterpret_cast<float4*>(arow) + q4 * 8;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) dst[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+              }
+              continue;
+            }
+          }
           uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
-          if constexpr (VARLEN) {
+          for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(f[2 * i], f[2 * i + 1]);
+          if constexpr (ROWSTORE) {
             if (store_row) {
               uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 64);
 #pragma unroll
@@ -1078,16 +1185,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(C::O_EMPTY + t));
-      if constexpr (!VARLEN) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::O_EMPTY + t));
+      if constexpr (!ROWSTORE) {
         fence_proxy_async_smem();
         mbar_arrive(bar(C::EPI + t));
       }
-      if (store_row) {
-        const float lse = (m_use + lg2(l)) * 0.69314718055994530942f;
-        p.lse[(size_t)un.b * p.lse_bs + (size_t)un.h * p.lse_hs + un.rb + row] = lse;
-      }
-      if constexpr (!VARLEN) {
+      if (store_row) p.lse[lse_at] = lse2 * 0.69314718055994530942f;
+      if constexpr (!ROWSTORE) {
         if (rit == 0) {
           // one thread stores the tile once all 128 rows are staged
           drain_wait(bar(C::EPI + t), e_use & 1u, limit);
@@ -1102,7 +1207,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       __syncwarp();
     }
-    if constexpr (!VARLEN) {
+    if constexpr (!ROWSTORE) {
       if (rit == 0) tma_store_wait_all();
     }
     __syncwarp();
@@ -1199,13 +1304,13 @@ fa_status check_device_ptr(const void* ptr, int device) {
 
 struct DeviceInfo {
   int sms = 0;
-  bool configured[8] = {false, false, false, false, false, false, false, false};
+  bool configured[12] = {};   // per kernel instantiation: shared-memory attribute set
 };
 
-template <int D, bool BF16, bool VARLEN>
+template <int D, bool BF16, int KIND>
 fa_status launch(const fa::Params& prm, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                  const CUtensorMap& o, int grid, bool* configured, cudaStream_t stream) {
-  auto kern = fa::fa_fwd_kernel<D, BF16, VARLEN>;
+  auto kern = fa::fa_fwd_kernel<D, BF16, KIND>;
   const int smem = fa::Cfg<D>::SMEM_BYTES;
   if (!*configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1265,18 +1370,28 @@ fa_status launch_units(fa::Params& prm, const CUtensorMap& mq, const CUtensorMap
     if (e != cudaSuccess) return cuda_fail((int)e);
   }
   bool* cfg = g_dev[dev].configured;
+  using fa::DENSE;
+  using fa::PACKED;
+  using fa::RING;
+  if (prm.nseg > 0) {
+    if (D == 128)
+      return dtype == FA_BF16 ? launch<128, true, RING>(prm, mq, mk, mv, mo, grid, &cfg[8], s)
+                              : launch<128, false, RING>(prm, mq, mk, mv, mo, grid, &cfg[9], s);
+    return dtype == FA_BF16 ? launch<64, true, RING>(prm, mq, mk, mv, mo, grid, &cfg[10], s)
+                            : launch<64, false, RING>(prm, mq, mk, mv, mo, grid, &cfg[11], s);
+  }
   if (prm.cu_q) {
     if (D == 128)
-      return dtype == FA_BF16 ? launch<128, true, true>(prm, mq, mk, mv, mo, grid, &cfg[4], s)
-                              : launch<128, false, true>(prm, mq, mk, mv, mo, grid, &cfg[5], s);
-    return dtype == FA_BF16 ? launch<64, true, true>(prm, mq, mk, mv, mo, grid, &cfg[6], s)
-                            : launch<64, false, true>(prm, mq, mk, mv, mo, grid, &cfg[7], s);
+      return dtype == FA_BF16 ? launch<128, true, PACKED>(prm, mq, mk, mv, mo, grid, &cfg[4], s)
+                              : launch<128, false, PACKED>(prm, mq, mk, mv, mo, grid, &cfg[5], s);
+    return dtype == FA_BF16 ? launch<64, true, PACKED>(prm, mq, mk, mv, mo, grid, &cfg[6], s)
+                            : launch<64, false, PACKED>(prm, mq, mk, mv, mo, grid, &cfg[7], s);
   }
   if (D == 128)
-    return dtype == FA_BF16 ? launch<128, true, false>(prm, mq, mk, mv, mo, grid, &cfg[0], s)
-                            : launch<128, false, false>(prm, mq, mk, mv, mo, grid, &cfg[1], s);
-  return dtype == FA_BF16 ? launch<64, true, false>(prm, mq, mk, mv, mo, grid, &cfg[2], s)
-                          : launch<64, false, false>(prm, mq, mk, mv, mo, grid, &cfg[3], s);
+    return dtype == FA_BF16 ? launch<128, true, DENSE>(prm, mq, mk, mv, mo, grid, &cfg[0], s)
+                            : launch<128, false, DENSE>(prm, mq, mk, mv, mo, grid, &cfg[1], s);
+  return dtype == FA_BF16 ? launch<64, true, DENSE>(prm, mq, mk, mv, mo, grid, &cfg[2], s)
+                          : launch<64, false, DENSE>(prm, mq, mk, mv, mo, grid, &cfg[3], s);
 }
 
 // Heads whose K and V (Sk keys each) fit together in about 48 MB of L2.
@@ -1369,7 +1484,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* 
   if ((st = make_map(&mv, v, dtype, layout, B, H, Sk, D)) != FA_OK) return st;
   if ((st = make_map(&mo, o, dtype, layout, B, H, Sq, D)) != FA_OK) return st;
 
-  fa::Params prm;
+  fa::Params prm{};   // no ring segments
   prm.lse = lse;
   prm.cu_q = nullptr;
   prm.cu_k = nullptr;
@@ -1631,13 +1746,16 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
   if ((st = make_map(&mv, v, dtype, FA_BSND, 1, H, total_k, D)) != FA_OK) return st;
   if ((st = make_map(&mo, o, dtype, FA_BSND, 1, H, total_q, D)) != FA_OK) return st;
 
-  fa::Params prm;
+  fa::Params prm{};   // no ring segments
   prm.lse = lse;
   prm.cu_q = cu_seqlens_q;
   prm.cu_k = cu_seqlens_k;
   prm.total_q = (int)total_q;
   prm.total_k = (int)total_k;
   prm.o = static_cast<uint8_t*>(o);
+  prm.o_bs = 0;                 // row r of head h at (r * H + h) * D
+  prm.o_hs = D;
+  prm.o_rs = H * D;
   prm.lse_bs = 0;
   prm.lse_hs = total_q;
   prm.B = (int)B;
@@ -1656,6 +1774,105 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
   prm.wait_limit_ns = 1000000000ull;
   prm.withhold_loads = 0;
   set_softmax_params(prm, SoftmaxOpts());
+  return launch_units(prm, mq, mk, mv, mo, D, dtype, static_cast<unsigned int*>(workspace), dev, sms, stream);
+}
+
+fa_status fa_fwd_ring_step(const void* q, const void* k, const void* v, void* o, float* acc, float* lse, int64_t B,
+                            int64_t H, int64_t Sq, int64_t Sk, int64_t D, int64_t rows, const fa_ring_segment* segs,
+                            int nseg, fa_layout layout, float scale, fa_dtype dtype, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  bool noop = false;
+  fa_status hst = host_checks(q, k, v, o, lse, B, H, Sq, Sk, D, layout, scale, dtype, &noop);
+  if (hst != FA_OK) return hst;
+  if (!segs || nseg < 1 || nseg > 2 || rows < 0 || rows > Sq) return FA_ERR_INVALID_ARG;
+  if (noop || rows == 0) return FA_OK;
+  bool need_acc = false;
+  for (int s = 0; s < nseg; ++s) {
+    const fa_ring_segment& g = segs[s];
+    if (g.row0 < 0 || g.row0 > Sq - rows || g.key0 < 0 || g.keys < 1 || g.key0 > Sk - g.keys) return FA_ERR_INVALID_ARG;
+    if ((g.first != 0 && g.first != 1) || (g.last != 0 && g.last != 1)) return FA_ERR_INVALID_ARG;
+    if (g.causal_offset >= ((int64_t)1 << 30)) return FA_ERR_UNSUPPORTED;
+    if (!g.first || !g.last) need_acc = true;
+  }
+  if (nseg == 2 && segs[0].row0 < segs[1].row0 + rows && segs[1].row0 < segs[0].row0 + rows)
+    return FA_ERR_INVALID_ARG;   // two segments would write the same rows
+  if (!workspace || workspace_bytes < kWorkspaceBytes) return FA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) & 15u) return FA_ERR_MISALIGNED;
+  if (need_acc && !acc) return FA_ERR_INVALID_ARG;
+  if (acc && (reinterpret_cast<uintptr_t>(acc) & 15u)) return FA_ERR_MISALIGNED;
+  const size_t qbytes = (size_t)(B * H * Sq * D) * 2, kvbytes = (size_t)(B * H * Sk * D) * 2;
+  const size_t lbytes = (size_t)(B * H * Sq) * 4, abytes = (size_t)(B * H * Sq * D) * 4;
+  {
+    const void* bufs[7] = {q, k, v, o, lse, acc, workspace};
+    const size_t sizes[7] = {qbytes, kvbytes, kvbytes, qbytes, lbytes, abytes, workspace_bytes};
+    for (int i = 5; i < 7; ++i)   // acc and the workspace against every other buffer
+      for (int j = 0; j < 7; ++j)
+        if (i != j && bufs[i] && bufs[j] && overlaps(bufs[i], sizes[i], bufs[j], sizes[j])) return FA_ERR_ALIAS;
+  }
+
+  int dev = 0, sms = 0;
+  const void* ptrs[7] = {q, k, v, o, lse, acc, workspace};
+  fa_status st = device_checks(ptrs, 7, &dev, &sms);
+  if (st != FA_OK) return st;
+  CUtensorMap mq, mk, mv, mo;
+  if ((st = make_map(&mq, q, dtype, layout, B, H, Sq, D)) != FA_OK) return st;
+  if ((st = make_map(&mk, k, dtype, layout, B, H, Sk, D)) != FA_OK) return st;
+  if ((st = make_map(&mv, v, dtype, layout, B, H, Sk, D)) != FA_OK) return st;
+  if ((st = make_map(&mo, o, dtype, layout, B, H, Sq, D)) != FA_OK) return st;
+
+  // the segment with more keys first: its units are the longer ones
+  int order[2] = {0, 1};
+  if (nseg == 2 && segs[1].keys > segs[0].keys) {
+    order[0] = 1;
+    order[1] = 0;
+  }
+  int64_t max_keys = 0;
+  for (int s = 0; s < nseg; ++s) max_keys = segs[s].keys > max_keys ? segs[s].keys : max_keys;
+  const int64_t nqb = (rows + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+  if (nseg * B * H * nqb >= ((int64_t)1 << 30)) return FA_ERR_UNSUPPORTED;
+
+  fa::Params prm{};
+  prm.lse = lse;
+  prm.o = static_cast<uint8_t*>(o);
+  if (layout == FA_BHSD) {
+    prm.o_bs = H * Sq * D;
+    prm.o_hs = Sq * D;
+    prm.o_rs = D;
+  } else {
+    prm.o_bs = Sq * H * D;
+    prm.o_hs = D;
+    prm.o_rs = H * D;
+  }
+  prm.lse_bs = H * Sq;
+  prm.lse_hs = Sq;
+  prm.B = (int)B;
+  prm.H = (int)H;
+  prm.Sq = (int)rows;
+  prm.Sk = (int)max_keys;
+  prm.nqb = (int)nqb;
+  prm.tk = (int)((max_keys + fa::BN - 1) / fa::BN);
+  prm.bh = (int)(B * H);
+  prm.head0 = 0;
+  prm.group_heads = l2_group_heads(max_keys, D, B * H);
+  prm.total_units = (int)(nseg * B * H * nqb);
+  prm.causal = 0;
+  prm.bhsd = layout == FA_BHSD ? 1 : 0;
+  prm.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  prm.wait_limit_ns = 1000000000ull;
+  prm.withhold_loads = 0;
+  set_softmax_params(prm, SoftmaxOpts());
+  prm.nseg = nseg;
+  prm.seg_units0 = (int)(B * H * nqb);
+  for (int i = 0; i < nseg; ++i) {
+    const fa_ring_segment& g = segs[order[i]];
+    prm.seg_row0[i] = (int)g.row0;
+    prm.seg_key0[i] = (int)g.key0;
+    prm.seg_sk[i] = (int)g.keys;
+    prm.seg_causal[i] = g.causal_offset >= 0 ? 1 : 0;
+    prm.seg_coff[i] = g.causal_offset >= 0 ? (int)g.causal_offset : 0;
+    prm.seg_flags[i] = (g.first ? 1 : 0) | (g.last ? 2 : 0);
+  }
+  prm.acc = acc;
   return launch_units(prm, mq, mk, mv, mo, D, dtype, static_cast<unsigned int*>(workspace), dev, sms, stream);
 }
 

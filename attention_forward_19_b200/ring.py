@@ -17,17 +17,23 @@ is that split for self-attention (Sq = Sk = S):
 * For every (query chunk, key chunk) pair the key chunk is either entirely
   visible (an earlier chunk, or no mask), the diagonal block (the same chunk:
   the causal mask within it is exactly the top-left mask of fa_fwd), or
-  entirely masked (a later chunk: skipped).  Each visible block is one fa_fwd
-  call; its normalised partial (O, LSE) is merged into a running fp32 result
-  by fa_lse_merge, and the last merge writes the output in the input dtype.
+  entirely masked (a later chunk: skipped).
+* A step's blocks form at most one "segment" per query chunk: the query chunk
+  against a run of consecutive held key chunks, of which only the last may be
+  the diagonal block (a causal mask offset by the full chunks before it).
+  All segments of a step run as ONE launch of fa_fwd_ring_step, which merges
+  each segment's result into the running result of its rows in the attention
+  epilogue (fp32 O in a buffer, the LSE in the output LSE) and writes the
+  output in the input dtype at the rows' last segment.
 
-Local tensors are chunk-major so that every chunk is contiguous: q, k, v of a
-rank are [n, B, Sc, H, D] (layout "BSND") or [n, B, H, Sc, D] ("BHSD") with n
-chunks of Sc rows, and the LSE is [n, B, H, Sc].  shard() and unshard() convert
-from and to whole-sequence tensors.
+Local tensors hold a rank's chunks concatenated along the sequence axis, in
+the order of chunk_ids_of: q, k, v of a rank are [B, n * Sc, H, D] (layout
+"BSND") or [B, H, n * Sc, D] ("BHSD"), and the LSE is [B, H, n * Sc].
+shard() and unshard() convert from and to whole-sequence tensors.
 
-The per-block compute and merge are plain callables, so the schedule and the
-exchange can be run on the CPU with other implementations of those two steps.
+The step is a plain callable, so the schedule and the exchange can also run on
+the CPU with the step composed of other implementations of block attention and
+the merge (BlockwiseStep).
 """
 import math
 
@@ -91,53 +97,137 @@ def _seq_dim(layout):
 
 
 def shard(x, rank, world, layout, chunk_ids_of=zigzag_chunk_ids):
-    """This rank's chunks of a whole-sequence tensor [B, S, H, D] / [B, H, S, D], chunk-major."""
+    """This rank's rows of a whole-sequence tensor [B, S, H, D] / [B, H, S, D]: its chunks concatenated
+    along the sequence axis in chunk_ids_of order."""
     dim = _seq_dim(layout)
     S = x.shape[dim]
     if S % (2 * world):
         raise ValueError(f"sequence length {S} is not a multiple of 2 * world = {2 * world}")
     chunks = x.chunk(2 * world, dim=dim)
-    return torch.stack([chunks[c] for c in chunk_ids_of(rank, world)]).contiguous()
+    return torch.cat([chunks[c] for c in chunk_ids_of(rank, world)], dim=dim).contiguous()
 
 
 def unshard(parts, layout, chunk_ids_of=zigzag_chunk_ids, seq_dim=None):
-    """Whole-sequence tensor from every rank's chunk-major part (parts[r] of rank r).
+    """Whole-sequence tensor from every rank's part (parts[r] of rank r, as shard() gives it).
 
-    seq_dim: the sequence axis of one chunk (default from the layout; 2 for the LSE [B, H, Sc])."""
+    seq_dim: the sequence axis (default from the layout; 2 for the LSE [B, H, S])."""
     world = len(parts)
     dim = _seq_dim(layout) if seq_dim is None else seq_dim
     by_id = {}
     for r, p in enumerate(parts):
-        for i, c in enumerate(chunk_ids_of(r, world)):
-            by_id[c] = p[i]
+        ids = chunk_ids_of(r, world)
+        for c, piece in zip(ids, p.chunk(len(ids), dim=dim)):
+            by_id[c] = piece
     return torch.cat([by_id[c] for c in range(2 * world)], dim=dim)
+
+
+def step_plan(rank, world, causal, chunk_ids_of=zigzag_chunk_ids):
+    """The segments rank computes at each step: plan[t] = [(i, j_lo, j_hi, diagonal, first, last), ...].
+
+    Segment (i, j_lo, j_hi, ...) is local query chunk i against held key chunks j_lo .. j_hi - 1, all
+    entirely visible except the last when `diagonal`; first / last: the segment holds the first / the
+    last contributing block of chunk i.  A step's blocks for one query chunk that do not form such a
+    run become several segments (none do for the zigzag assignment)."""
+    plan = [[] for _ in range(world)]
+    for i, blocks in enumerate(contribution_plan(rank, world, causal, chunk_ids_of)):
+        by_step = {}
+        for (t, j, diag, first, last) in blocks:
+            by_step.setdefault(t, []).append((j, diag, first, last))
+        for t, bl in sorted(by_step.items()):
+            bl.sort()
+            run = [bl[0]]
+            for b in bl[1:]:
+                if b[0] == run[-1][0] + 1 and not run[-1][1]:
+                    run.append(b)
+                else:
+                    plan[t].append((i, run[0][0], run[-1][0] + 1, run[-1][1], run[0][2], run[-1][3]))
+                    run = [b]
+            plan[t].append((i, run[0][0], run[-1][0] + 1, run[-1][1], run[0][2], run[-1][3]))
+    return plan
 
 
 # ----------------------------------------------------------------------------- the two compute steps
 
 
-class CudaBlockOps:
-    """The block attention (fa_fwd) and the merge (fa_lse_merge) through the C ABI."""
+def fa_segments(segments, Sc):
+    """fa_fwd_ring_step segments (row0, key0, keys, causal_offset, first, last) of a step's segments:
+    local query chunk i is rows [i Sc, (i + 1) Sc); held key chunks j_lo .. j_hi - 1 are keys
+    [j_lo Sc, j_hi Sc); a diagonal last chunk is the causal mask offset by the full chunks before it."""
+    return [(i * Sc, j_lo * Sc, (j_hi - j_lo) * Sc, (j_hi - 1 - j_lo) * Sc if diag else -1, int(first), int(last))
+            for (i, j_lo, j_hi, diag, first, last) in segments]
 
-    acc_dtype = torch.float32      # the running result
-    lse_dtype = torch.float32      # what fa_fwd and fa_lse_merge write
+
+def launch_batches(segments):
+    """The step's segments in launches of at most two, no query chunk twice in one launch (in order)."""
+    batches, pending = [], list(segments)
+    while pending:
+        batch, used, rest = [], set(), []
+        for g in pending:
+            if g[0] in used or len(batch) == 2:
+                rest.append(g)
+            else:
+                batch.append(g)
+                used.add(g[0])
+        batches.append(batch)
+        pending = rest
+    return batches
+
+
+def _chunk(t, dim, i, Sc):
+    return t.narrow(dim, i * Sc, Sc)
+
+
+class CudaStepOps:
+    """A step's segments through fa_fwd_ring_step: one launch per step (segments of one query chunk
+    that a step splits further go to further launches)."""
+
+    acc_dtype = torch.float32      # the running O
+    lse_dtype = torch.float32      # the running and final LSE
 
     def __init__(self, layout, scale):
-        from . import flash_attention_forward, lse_merge, fa_fwd_workspace_size
+        from . import ring_step, fa_fwd_workspace_size
         self.layout, self.scale = layout, scale
-        self._fwd, self._merge = flash_attention_forward, lse_merge
+        self._step = ring_step
         self._ws_bytes = fa_fwd_workspace_size()
         self._ws = None
+        self.launches = 0
 
-    def block(self, q, k, v, diagonal, o, lse):
+    def step(self, q, k, v, segments, Sc, out, lse, acc):
         if self._ws is None or self._ws.device != q.device:
             self._ws = torch.empty(self._ws_bytes, dtype=torch.uint8, device=q.device)
-        self._fwd(q, k, v, layout=self.layout, causal=bool(diagonal), scale=self.scale, out=o, lse=lse,
-                  workspace=self._ws)
+        for batch in launch_batches(segments):
+            self._step(q, k, v, fa_segments(batch, Sc), Sc, out, lse, acc=acc, layout=self.layout,
+                       scale=self.scale, workspace=self._ws)
+            self.launches += 1
 
-    def merge(self, o_part, lse_part, o_acc, lse_acc, o_out, lse_out, accumulate, final):
-        self._merge(o_part, lse_part, o_acc, lse_acc, out=o_out, lse_out=lse_out, layout=self.layout,
-                    accumulate=accumulate, final=final)
+
+class BlockwiseStep:
+    """A step composed of block attention and the merge of partial results, block by block:
+    block(q, k, v, diagonal, o, lse) writes one block's normalised result, and
+    merge(o_part, lse_part, o_acc, lse_acc, o_out, lse_out, accumulate, final) merges it into the
+    running result.  The running LSE is kept in the output LSE, as fa_fwd_ring_step keeps it."""
+
+    def __init__(self, block_ops):
+        self.ops = block_ops
+        self.layout = block_ops.layout
+        self.acc_dtype, self.lse_dtype = block_ops.acc_dtype, block_ops.lse_dtype
+
+    def step(self, q, k, v, segments, Sc, out, lse, acc):
+        dim = _seq_dim(self.layout)
+        for (i, j_lo, j_hi, diag, first, last) in segments:
+            q_i, o_i, a_i = (_chunk(t, dim, i, Sc) for t in (q, out, acc if acc is not None else out))
+            l_i = _chunk(lse, 2, i, Sc)
+            for j in range(j_lo, j_hi):
+                d = diag and j == j_hi - 1
+                f = first and j == j_lo
+                z = last and j == j_hi - 1
+                if f and z:   # a single block: its result is the output
+                    self.ops.block(q_i, _chunk(k, dim, j, Sc), _chunk(v, dim, j, Sc), d, o_i, l_i)
+                    continue
+                part = torch.empty(q_i.shape, dtype=q.dtype, device=q.device)
+                part_lse = torch.empty(l_i.shape, dtype=self.lse_dtype, device=q.device)
+                self.ops.block(q_i, _chunk(k, dim, j, Sc), _chunk(v, dim, j, Sc), d, part, part_lse)
+                self.ops.merge(part, part_lse, a_i, l_i, o_i, l_i, accumulate=not f, final=z)
 
 
 # ----------------------------------------------------------------------------- exchanges
@@ -199,43 +289,33 @@ class LocalExchange:
 
 
 def ring_steps(q, k, v, rank, world, exchange, ops, causal, chunk_ids_of=zigzag_chunk_ids):
-    """Runs one rank's part of ring attention; returns (o like q, lse [n, B, H, Sc]).
+    """Runs one rank's part of ring attention; returns (o like q, lse [B, H, n * Sc]).
 
-    q, k, v: this rank's chunk-major tensors.  exchange: post(step, k, v) / wait(handle) giving
-    the next step's chunks.  ops: block(q, k, v, diagonal, o, lse) and merge(...), acc_dtype."""
+    q, k, v: this rank's local tensors (shard()).  exchange: post(step, k, v) / wait(handle) giving the
+    next step's chunks.  ops: step(q, k, v, segments, Sc, out, lse, acc) (CudaStepOps or BlockwiseStep),
+    acc_dtype, lse_dtype, layout."""
     if q.shape != k.shape or k.shape != v.shape:
-        raise ValueError("ring attention here is self-attention: q, k and v chunks must have one shape")
-    n = q.shape[0]
-    if n != len(chunk_ids_of(rank, world)):
-        raise ValueError(f"expected {len(chunk_ids_of(rank, world))} chunks, got {n}")
+        raise ValueError("ring attention here is self-attention: q, k and v must have one shape")
+    n = len(chunk_ids_of(rank, world))
     layout = ops.layout
+    dim = _seq_dim(layout)
     if layout == "BSND":
-        B, Sc, H, _ = q.shape[1:]
+        B, S_loc, H, _ = q.shape
     else:
-        B, H, Sc, _ = q.shape[1:]
-    plan = contribution_plan(rank, world, causal, chunk_ids_of)
+        B, H, S_loc, _ = q.shape
+    if S_loc % n:
+        raise ValueError(f"{S_loc} local rows do not split into {n} chunks")
+    Sc = S_loc // n
+    plan = step_plan(rank, world, causal, chunk_ids_of)
     out = torch.empty_like(q)
-    lse = torch.empty((n, B, H, Sc), dtype=ops.lse_dtype, device=q.device)
-    needs_merge = any(len(p) > 1 for p in plan)
-    if needs_merge:
-        acc = torch.empty(q.shape, dtype=ops.acc_dtype, device=q.device)
-        acc_lse = torch.empty((n, B, H, Sc), dtype=ops.acc_dtype, device=q.device)
-        part = torch.empty_like(q[0])
-        part_lse = torch.empty((B, H, Sc), dtype=ops.lse_dtype, device=q.device)
-    by_step = [[[] for _ in range(n)] for _ in range(world)]
-    for i, blocks in enumerate(plan):
-        for (t, j, diag, first, last) in blocks:
-            by_step[t][i].append((j, diag, first, last))
+    lse = torch.empty((B, H, S_loc), dtype=ops.lse_dtype, device=q.device)
+    needs_acc = any(not (g[4] and g[5]) for segs in plan for g in segs)
+    acc = torch.empty(q.shape, dtype=ops.acc_dtype, device=q.device) if needs_acc else None
     cur_k, cur_v = k, v
     for t in range(world):
         handle = exchange.post(t, cur_k, cur_v)
-        for i in range(n):
-            for (j, diag, first, last) in by_step[t][i]:
-                if first and last:       # a single block: its result is the output
-                    ops.block(q[i], cur_k[j], cur_v[j], diag, out[i], lse[i])
-                    continue
-                ops.block(q[i], cur_k[j], cur_v[j], diag, part, part_lse)
-                ops.merge(part, part_lse, acc[i], acc_lse[i], out[i], lse[i], accumulate=not first, final=last)
+        if plan[t]:
+            ops.step(q, cur_k, cur_v, plan[t], Sc, out, lse, acc)
         if handle is not None:
             cur_k, cur_v = exchange.wait(handle)
     return out, lse
@@ -245,8 +325,8 @@ def ring_attention_forward(q, k, v, causal=False, scale=None, layout="BSND", gro
                            chunk_ids_of=zigzag_chunk_ids):
     """Ring attention over the ranks of `group` (torch.distributed, one GPU per rank).
 
-    q, k, v: this rank's chunk-major CUDA tensors (see shard()).  Returns (o, lse) for this
-    rank's query chunks: o like q, lse fp32 [n, B, H, Sc].  scale=None uses 1/sqrt(D)."""
+    q, k, v: this rank's local CUDA tensors (see shard()).  Returns (o, lse) for this rank's query
+    rows: o like q, lse fp32 [B, H, n * Sc].  scale=None uses 1/sqrt(D)."""
     import torch.distributed as dist
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[-1])
@@ -256,7 +336,7 @@ def ring_attention_forward(q, k, v, causal=False, scale=None, layout="BSND", gro
     else:
         rank, world = 0, 1
         exchange = LocalExchange(0, 1, [k], [v])
-    return ring_steps(q, k, v, rank, world, exchange, CudaBlockOps(layout, scale), causal, chunk_ids_of)
+    return ring_steps(q, k, v, rank, world, exchange, CudaStepOps(layout, scale), causal, chunk_ids_of)
 
 
 def ring_attention_emulated(q, k, v, world, causal=False, scale=None, layout="BSND",
@@ -264,11 +344,11 @@ def ring_attention_emulated(q, k, v, world, causal=False, scale=None, layout="BS
     """The ring schedule of `world` ranks run one rank after another on one device.
 
     q, k, v: whole-sequence tensors [B, S, H, D] / [B, H, S, D].  Returns whole-sequence (o, lse)
-    assembled from the virtual ranks' results: the same blocks and merges as the real ring, with
-    the transfers replaced by lookups (LocalExchange)."""
+    assembled from the virtual ranks' results: the same steps as the real ring, with the transfers
+    replaced by lookups (LocalExchange).  ops: a step implementation (default CudaStepOps)."""
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[-1])
-    ops = CudaBlockOps(layout, scale) if ops is None else ops
+    ops = CudaStepOps(layout, scale) if ops is None else ops
     qs = [shard(q, r, world, layout, chunk_ids_of) for r in range(world)]
     ks = [shard(k, r, world, layout, chunk_ids_of) for r in range(world)]
     vs = [shard(v, r, world, layout, chunk_ids_of) for r in range(world)]

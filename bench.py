@@ -31,8 +31,13 @@ over the N ranks (strong scaling; default workload bf16 BHSD B=1 H=8
 S=65536 D=128 causal), each rank holding its zigzag pair of chunks and
 passing key/value chunks on over NCCL point-to-point.  A step is the whole
 ring; the time is the max over ranks and the value the whole sequence's
-flops / that time.  With N = 1 the ring has one rank (its two chunks, three
-blocks and one merge).
+flops / that time.  Each rank runs one fa_fwd_ring_step launch per ring step
+(the step's blocks attended and merged in one kernel).  With N = 1 the ring
+has one rank (its two chunks: one launch).  --ring --emulate-ranks W on one
+GPU runs the schedule of W virtual ranks one after another (the transfers
+replaced by lookups) and reports each virtual rank's share of the flops over
+its own time; the value projects W GPUs as the whole sequence's flops over
+the slowest virtual rank's time.
 
 --proj times attention followed by its output projection (fa_fwd_proj:
 y = o w_o^T with E = H * D output features, w_o seeded N(0, 1/(H D))) on the
@@ -506,6 +511,10 @@ def run_ring(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = bench_workload(args)
+    if args.emulate_ranks:
+        if world != 1:
+            raise SystemExit("--emulate-ranks runs on one GPU")
+        return run_ring_emulated(args, w, dev)
     if w.Sq != w.Sk or w.Sq % (2 * world):
         raise SystemExit(f"--ring needs Sq == Sk and a multiple of {2 * world} rows")
     q, k, v = make_qkv(w)                       # the same whole sequence on every rank, then its shard
@@ -544,9 +553,7 @@ def run_ring(args, rank, world, local_rank):
         return None
     peaks, peak_kind = load_peaks()
     peak = float(peaks["bf16_tflops"])
-    plan = ring.contribution_plan(0, world, w.causal)
-    blocks = sum(len(p) for p in plan)
-    merges = sum(len(p) for p in plan if len(p) > 1)
+    launches = ring_launches(ring.step_plan(0, world, w.causal))
     cfg = workload_config(w, world)
     cfg.update({"global_batch": w.B, "parallelism": f"cp{world} (ring over NCCL point-to-point, zigzag chunks)"})
     return {
@@ -559,9 +566,60 @@ def run_ring(args, rank, world, local_rank):
                      "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
                                     if peak_kind == "measured" else "fallback 1590 TFLOP/s",
                      "note": "per-GPU share of the whole sequence's flops over the slowest rank's time"},
-        "gpu_launches": (blocks + merges) * args.steps,
-        "gpu_launches_note": f"rank 0 per step: {blocks} fa_fwd block launches and {merges} fa_lse_merge launches",
+        "gpu_launches": launches * args.steps,
+        "gpu_launches_note": f"rank 0 per step: {launches} fa_fwd_ring_step launches (one per ring step)",
         "clocks": clk,
+    }
+
+
+def ring_launches(plan):
+    """fa_fwd_ring_step launches of a rank's step plan."""
+    from attention_forward_19_b200 import ring
+    return sum(len(ring.launch_batches(segs)) for segs in plan)
+
+
+def run_ring_emulated(args, w, dev):
+    """--ring --emulate-ranks W on one GPU: each virtual rank's ring (K timed repetitions) in turn."""
+    import attention_forward_19_b200 as fa
+    from attention_forward_19_b200 import ring
+    W = args.emulate_ranks
+    if w.Sq != w.Sk or w.Sq % (2 * W):
+        raise SystemExit(f"--ring needs Sq == Sk and a multiple of {2 * W} rows")
+    q, k, v = make_qkv(w)
+    qs, ks, vs = ([ring.shard(t, r, W, w.layout).to(dev) for r in range(W)] for t in (q, k, v))
+    del q, k, v
+    stream = torch.cuda.current_stream(dev)
+    ops = ring.CudaStepOps(w.layout, w.scale)
+    per_rank = []
+    for r in range(W):
+        def step():
+            return ring.ring_steps(qs[r], ks[r], vs[r], r, W, ring.LocalExchange(r, W, ks, vs), ops, w.causal)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        plan = ring.contribution_plan(r, W, w.causal)
+        rank_flops = sum(w.flops() / (2 * W) ** 2 / (0.5 if w.causal else 1.0) * (0.5 if d else 1.0)
+                         for blocks in plan for (_, _, d, _, _) in blocks)
+        ms = e0.elapsed_time(e1) / args.steps
+        per_rank.append((ms, rank_flops / (ms * 1e-3) / 1e12))
+    fa.check_device_status(stream)
+    worst = max(ms for ms, _ in per_rank)
+    cfg = workload_config(w, 1)
+    cfg.update({"global_batch": w.B, "parallelism": f"cp{W} emulated on one GPU (zigzag chunks, no transfers)"})
+    return {
+        "metric": f"ring attn fwd TFLOP/s, {W} ranks emulated on one GPU (projected: whole sequence over the "
+                  f"slowest virtual rank)", "value": w.flops() / (worst * 1e-3) / 1e12, "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": worst, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": cfg,
+        "per_rank_ms": [round(ms, 4) for ms, _ in per_rank],
+        "per_rank_share_tflops": [round(t, 1) for _, t in per_rank],
+        "gpu_launches": ring_launches(ring.step_plan(0, W, w.causal)) * args.steps * W,
     }
 
 
@@ -699,6 +757,8 @@ def main():
     ap.add_argument("--atomic", action="store_true", help="with --backward: the non-deterministic variant")
     ap.add_argument("--ring", action="store_true", help="time ring attention of one sequence over the ranks")
     ap.add_argument("--proj", action="store_true", help="time attention + output projection (fa_fwd_proj)")
+    ap.add_argument("--emulate-ranks", type=int, default=0,
+                    help="with --ring on one GPU: time the schedule of this many virtual ranks")
     ap.add_argument("--strong", action="store_true",
                     help="split the workload itself across the ranks (default: weak scaling, one workload per rank)")
     ap.add_argument("--e2e-chunks", type=int, default=8,

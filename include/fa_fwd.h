@@ -44,7 +44,8 @@
  * fa_fwd_noalloc, fa_fwd_varlen) the library exports its backward pass
  * (fa_bwd, fa_bwd_atomic), the merge of
  * partial results that ring attention over several GPUs is built from
- * (fa_lse_merge), and the attention output projection (fa_out_proj,
+ * (fa_lse_merge), one ring step with that merge fused into the attention
+ * (fa_fwd_ring_step), and the attention output projection (fa_out_proj,
  * fa_fwd_proj).  Each is described at its declaration below.
  */
 #ifndef FA_FWD_H
@@ -405,6 +406,61 @@ enum { FA_MERGE_ACCUMULATE = 1, FA_MERGE_FINAL = 2 };
 fa_status fa_lse_merge(const void *o_part, const float *lse_part, float *o_acc, float *lse_acc,
                        void *o_out, float *lse_out, int64_t B, int64_t H, int64_t S, int64_t D,
                        fa_layout layout, fa_dtype dtype, int flags, void *stream);
+
+/*
+ * fa_fwd_ring_step -- one step of ring attention in one launch.  Ring
+ * attention (page "FlashAttention in ops-transformer on Ascend NPU"
+ * (ai6s.net/6a0d3bfb), section "what else is in the ops-transformer
+ * repository"; page "64K long-sequence FlashAttention" (ai6s.net/6a140d07),
+ * section "performance tuning tips", multi-card parallelism) gives each rank,
+ * at each step, one or two blocks of its query rows against the key/value
+ * chunks it holds at that step.  This call attends every such block (a
+ * "segment") and merges the result into the running result of its rows in
+ * the attention kernel's epilogue -- the update fa_lse_merge applies, without
+ * the partial result's round trip through memory:
+ *     LSE = log(exp(LSE_run) + exp(LSE_seg))
+ *     O   = exp(LSE_run - LSE) O_run + exp(LSE_seg - LSE) O_seg
+ *
+ * q, o     this rank's query rows and output: [B, Sq, H, D] (FA_BSND) or
+ *          [B, H, Sq, D] (FA_BHSD), fp16 / bf16, 16-byte aligned
+ * k, v     the key/value rows held at this step, Sk of them, same layout and
+ *          dtype, 16-byte aligned; read only
+ * lse      fp32 [B, H, Sq]: the running LSE (read where a segment has
+ *          first = 0) and the merged LSE (written for every segment row)
+ * acc      fp32 like o: the running O, read where first = 0 and written where
+ *          last = 0; may be NULL when every segment has first = last = 1.
+ *          16-byte aligned
+ * rows     query rows per segment (the same for every segment)
+ * segs     nseg (1 or 2) segments with disjoint row ranges; segment s covers
+ *          query rows [row0, row0 + rows) and keys [key0, key0 + keys) of
+ *          k / v.  causal_offset >= 0: key c of the segment (counted from
+ *          key0) is visible from its row r (counted from row0) iff
+ *          c <= r + causal_offset, so every row sees key 0; causal_offset < 0:
+ *          every key is visible.  first = 1: the rows have no earlier result
+ *          (acc and lse are not read); last = 1: the merged result is final
+ *          and written to o in the input dtype (rounded to nearest), else to
+ *          acc in fp32.
+ *
+ * The work is scheduled as one persistent launch over both segments' work
+ * units (longest first); workspace as for fa_fwd_ws (fa_fwd_workspace_size
+ * bytes, zeroed on `stream` by the call).  The caller owns every buffer;
+ * acc and the workspace must not overlap any other buffer, and o / lse none
+ * of the inputs (FA_ERR_ALIAS).  FA_ERR_INVALID_ARG for a segment outside
+ * the tensors, overlapping segments, flags other than 0 / 1, or a missing
+ * acc or workspace.  Other errors as for fa_fwd.  Asynchronous on `stream`.
+ */
+typedef struct fa_ring_segment {
+  int64_t row0;           /* first query row of q / o / lse */
+  int64_t key0;           /* first key row of k / v */
+  int64_t keys;           /* keys attended, >= 1 */
+  int64_t causal_offset;  /* < 0: no mask; >= 0: key c visible from row r iff c <= r + causal_offset */
+  int32_t first;          /* 1: no running result yet */
+  int32_t last;           /* 1: write the final output */
+} fa_ring_segment;
+fa_status fa_fwd_ring_step(const void *q, const void *k, const void *v, void *o, float *acc, float *lse,
+                           int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D, int64_t rows,
+                           const fa_ring_segment *segs, int nseg, fa_layout layout, float scale,
+                           fa_dtype dtype, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * fa_out_proj -- the attention output projection Y = O W^T (page "catlass

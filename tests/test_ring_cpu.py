@@ -18,45 +18,9 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 from attention_forward_19_b200 import ring
+from ring_oracle_ops import OracleOps
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-
-
-class OracleOps:
-    """Block attention and merge from the oracle, in fp64 on the CPU."""
-
-    acc_dtype = torch.float64
-    lse_dtype = torch.float64
-
-    def __init__(self, layout, scale):
-        from oracle import attn as oracle_attn
-        self.layout, self.scale, self.orc = layout, scale, oracle_attn.default()
-        self.calls = []
-
-    def _to_layout(self, o_bhsd):
-        t = torch.from_numpy(o_bhsd)
-        return t.permute(0, 2, 1, 3) if self.layout == "BSND" else t
-
-    def _head_major(self, t):
-        return (t.permute(0, 2, 1, 3) if self.layout == "BSND" else t).double().numpy()
-
-    def block(self, q, k, v, diagonal, o, lse):
-        self.calls.append(bool(diagonal))
-        oo, ll = self.orc.fwd(q, k, v, layout=self.layout, causal=bool(diagonal), scale=self.scale)
-        o.copy_(self._to_layout(oo))
-        lse.copy_(torch.from_numpy(ll))
-
-    def merge(self, o_part, lse_part, o_acc, lse_acc, o_out, lse_out, accumulate, final):
-        from oracle.merge import merge_partials
-        parts = [self._head_major(o_part)]
-        lses = [lse_part.double().numpy()]
-        if accumulate:
-            parts.insert(0, self._head_major(o_acc))
-            lses.insert(0, lse_acc.double().numpy())
-        o, l = merge_partials(parts, lses)
-        dst_o, dst_l = (o_out, lse_out) if final else (o_acc, lse_acc)
-        dst_o.copy_(self._to_layout(o))
-        dst_l.copy_(torch.from_numpy(l))
 
 
 def _qkv(layout, B=1, H=2, S=48, D=16, seed=5):
@@ -106,6 +70,53 @@ def test_every_visible_key_is_used_exactly_once(world, causal):
     assert np.array_equal(count, mask)
 
 
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("causal", [False, True])
+def test_step_segments_cover_every_visible_key_exactly_once(world, causal):
+    # the fa_fwd_ring_step segments of every rank and step, expanded to (global row, global key) pairs
+    Sc = 3
+    S = 2 * world * Sc
+    count = np.zeros((S, S), dtype=int)
+    for r in range(world):
+        mine = ring.zigzag_chunk_ids(r, world)
+        for t, segs in enumerate(ring.step_plan(r, world, causal)):
+            held = ring.zigzag_chunk_ids(ring.ring_source(r, world, t), world)
+            for (row0, key0, keys, off, _, _) in ring.fa_segments(segs, Sc):
+                for rr in range(Sc):
+                    grow = mine[(row0 + rr) // Sc] * Sc + (row0 + rr) % Sc
+                    for c in range(keys):
+                        if off >= 0 and c > rr + off:
+                            continue
+                        count[grow, held[(key0 + c) // Sc] * Sc + (key0 + c) % Sc] += 1
+    mask = np.tril(np.ones((S, S), dtype=int)) if causal else np.ones((S, S), dtype=int)
+    assert np.array_equal(count, mask)
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("causal", [False, True])
+def test_step_plan_first_and_last_and_one_launch_per_step(world, causal):
+    for r in range(world):
+        plan = ring.step_plan(r, world, causal)
+        for i in range(2):
+            seq = [g for segs in plan for g in segs if g[0] == i]
+            assert seq and seq[0][4] and seq[-1][5]
+            assert sum(g[4] for g in seq) == 1 and sum(g[5] for g in seq) == 1
+        for segs in plan:
+            # zigzag: at most one segment per query chunk, so each step is one launch
+            assert len({g[0] for g in segs}) == len(segs) <= 2
+            assert len(ring.launch_batches(segs)) == (1 if segs else 0)
+            # only a segment's last key chunk may be the diagonal block, and keys start at chunk 0
+            assert all(g[1] == 0 and g[2] in (1, 2) for g in segs)
+    # with causal zigzag chunks every step has work on every rank
+    if causal:
+        assert all(ring.step_plan(r, world, True)[t] for r in range(world) for t in range(world))
+
+
+def test_launch_batches_split_repeated_query_chunks():
+    segs = [(0, 0, 1, False, True, False), (0, 1, 2, False, False, True), (1, 0, 2, True, True, True)]
+    assert ring.launch_batches(segs) == [[segs[0], segs[2]], [segs[1]]]
+
+
 def test_zigzag_balances_causal_work():
     world = 4
     work = []
@@ -119,7 +130,10 @@ def test_zigzag_balances_causal_work():
 def test_shard_unshard_round_trip(layout):
     x = _qkv(layout, S=24)[0]
     parts = [ring.shard(x, r, 3, layout) for r in range(3)]
-    assert all(p.is_contiguous() and p.shape[0] == 2 for p in parts)
+    dim = 1 if layout == "BSND" else 2
+    assert all(p.is_contiguous() and p.shape[dim] == 8 for p in parts)      # two chunks of 4 rows
+    # rank 1 holds chunks 1 and 4, in that order
+    assert torch.equal(parts[1], torch.cat([x.narrow(dim, 4, 4), x.narrow(dim, 16, 4)], dim=dim))
     assert torch.equal(ring.unshard(parts, layout), x)
     with pytest.raises(ValueError):
         ring.shard(x, 0, 5, layout)            # 24 rows are not a multiple of 10
@@ -135,7 +149,8 @@ def test_emulated_ring_with_oracle_steps_matches_whole_attention(world, causal, 
     q, k, v = _qkv(layout, S=2 * world * 6)
     scale = 0.3
     ops = OracleOps(layout, scale)
-    o, l = ring.ring_attention_emulated(q, k, v, world, causal=causal, scale=scale, layout=layout, ops=ops)
+    o, l = ring.ring_attention_emulated(q, k, v, world, causal=causal, scale=scale, layout=layout,
+                                        ops=ring.BlockwiseStep(ops))
     o_ref, l_ref = _oracle_whole(q, k, v, layout, causal, scale)
     assert float((o - o_ref).abs().max()) < 1e-12
     assert float((l - l_ref).abs().max()) < 1e-12
@@ -163,7 +178,7 @@ def _gloo_worker(rank, world, port, layout, causal, out):
         from attention_forward_19_b200 import ring as ring_mod
         q, k, v = _qkv(layout, S=2 * world * 5)
         mine = [ring_mod.shard(t, rank, world, layout) for t in (q, k, v)]
-        ops = OracleOps(layout, 0.25)
+        ops = ring_mod.BlockwiseStep(OracleOps(layout, 0.25))
         o, l = ring_mod.ring_steps(*mine, rank, world, ring_mod.P2PExchange(), ops, causal)
         out[rank] = (o.numpy(), l.numpy())
         dist.barrier()
@@ -213,7 +228,7 @@ def _gloo_subgroup_worker(rank, world, port, out):
             assert (ex.rank, ex.world) == (grank, 2)
             # the peers are named by their global ranks: the other member, in both directions
             assert ex.next == ex.prev == members[1 - grank]
-            o, l = ring_mod.ring_steps(*mine, grank, 2, ex, OracleOps("BHSD", 0.25), True)
+            o, l = ring_mod.ring_steps(*mine, grank, 2, ex, ring_mod.BlockwiseStep(OracleOps("BHSD", 0.25)), True)
             out[grank] = (o.numpy(), l.numpy())
         dist.barrier()
     finally:

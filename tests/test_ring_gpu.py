@@ -5,9 +5,15 @@
   row counts, including rows whose LSE is -inf.  The kernel works in fp32:
   bound 1e-5 relative for the running result and the LSE, and, for the 16-bit
   output, one unit in the last place of the output type.
-* The ring schedule of W ranks emulated on one GPU (the same fa_fwd blocks and
-  fa_lse_merge merges as the distributed run; only the transfers are replaced
-  by lookups) against whole-sequence attention from the fp64 oracle, with the
+* fa_fwd_ring_step (a ring step's blocks attended and merged in one launch)
+  against the same step composed of oracle blocks and oracle merges in fp64
+  (ring.BlockwiseStep), over several steps: causal masks offset by whole
+  chunks, a segment starting at a later key chunk, first / last flags, the
+  running result (fp32 O and LSE) after a step and the final output, ragged
+  chunk sizes, D = 64 and 128, both dtypes and layouts.
+* The ring schedule of W ranks emulated on one GPU (the same fa_fwd_ring_step
+  launches as the distributed run; only the transfers are replaced by
+  lookups) against whole-sequence attention from the fp64 oracle, with the
   forward's bounds: max |O - O_oracle| <= 2e-2 (bf16) / 1e-2 (fp16), max
   |LSE - LSE_oracle| <= 1e-3.  Chunk sizes include ragged ones (not multiples
   of 128 rows), and the 64K-row, 8-head causal workload split over 8 ranks is
@@ -22,6 +28,7 @@ import torch
 import attention_forward_19_b200 as fa
 from attention_forward_19_b200 import ring
 from oracle.merge import merge_partials
+from ring_oracle_ops import OracleOps
 
 pytestmark = pytest.mark.gpu
 
@@ -92,6 +99,86 @@ def _qkv(layout, dtype, B, H, S, D, seed, std=1.0):
     g = torch.Generator().manual_seed(seed)
     shape = (B, S, H, D) if layout == "BSND" else (B, H, S, D)
     return [(torch.randn(shape, generator=g) * (std if i < 2 else 1.0)).to(dtype) for i in range(3)]
+
+
+STEP_CASES = [
+    # layout, dtype, B, H, Sc (rows per chunk), D
+    ("BHSD", torch.bfloat16, 1, 2, 200, 128),
+    ("BSND", torch.float16, 2, 2, 129, 64),
+    ("BSND", torch.bfloat16, 1, 3, 256, 128),
+    ("BHSD", torch.float16, 1, 1, 40, 128),
+]
+
+# three steps over two local query chunks (segments: query chunk, key chunks [lo, hi), diagonal last
+# chunk, first, last): diagonal blocks with causal offsets 0 and Sc; a full two-chunk segment merged
+# into a running result; a segment from the second key chunk with its diagonal; the final merges
+STEPS = [
+    [(0, 0, 1, True, True, False), (1, 0, 2, True, True, False)],
+    [(1, 0, 2, False, False, False), (0, 1, 2, True, False, True)],
+    [(1, 0, 1, False, False, True)],
+]
+
+
+@pytest.mark.parametrize("case", STEP_CASES, ids=lambda c: f"{c[0]}_{str(c[1])[6:]}_B{c[2]}H{c[3]}_Sc{c[4]}_D{c[5]}")
+def test_ring_step_matches_oracle_blocks_and_merges(case):
+    _need_gpu()
+    layout, dtype, B, H, Sc, D = case
+    scale = 1.0 / math.sqrt(D)
+    g = torch.Generator().manual_seed(Sc * 7 + D)
+    shape = (B, 2 * Sc, H, D) if layout == "BSND" else (B, H, 2 * Sc, D)
+    q = torch.randn(shape, generator=g).to(dtype)
+    kvs = [[torch.randn(shape, generator=g).to(dtype) for _ in range(2)] for _ in STEPS]
+    ref = ring.BlockwiseStep(OracleOps(layout, scale))
+    r_out, r_lse, r_acc = (torch.zeros(shape, dtype=torch.float64), torch.zeros((B, H, 2 * Sc), dtype=torch.float64),
+                           torch.zeros(shape, dtype=torch.float64))
+    ops = ring.CudaStepOps(layout, scale)
+    qd = q.cuda()
+    out = torch.full(shape, float("nan"), dtype=dtype, device="cuda")
+    lse = torch.full((B, H, 2 * Sc), float("nan"), device="cuda")
+    acc = torch.full(shape, float("nan"), device="cuda")
+    seq = 1 if layout == "BSND" else 2
+    for n, (segs, (k, v)) in enumerate(zip(STEPS, kvs)):
+        ops.step(qd, k.cuda(), v.cuda(), segs, Sc, out, lse, acc)
+        ref.step(q.double(), k.double(), v.double(), segs, Sc, r_out, r_lse, r_acc)
+        fa.check_device_status()
+        if n == 0:
+            # after the first step both chunks hold running results: fp32 O in acc, LSE in lse
+            err_o = float((acc.double().cpu() - r_acc).abs().max())
+            err_l = float((lse.double().cpu() - r_lse).abs().max())
+            assert err_o <= O_TOL[dtype] and err_l <= LSE_TOL, (err_o, err_l)
+            assert torch.isnan(out).all()          # nothing final yet
+    err_o = float((out.double().cpu() - r_out).abs().max())
+    err_l = float((lse.double().cpu() - r_lse).abs().max())
+    print(f"PARITY ring step {layout} {dtype} B{B} H{H} Sc{Sc} D{D}: max|dO| {err_o:.3e} max|dLSE| {err_l:.3e}")
+    assert err_o <= O_TOL[dtype] and err_l <= LSE_TOL
+    assert ops.launches == len(STEPS)
+
+
+def test_ring_step_rejects_bad_segments():
+    _need_gpu()
+    shape = (1, 256, 2, 128)
+    q, k, v, out = (torch.zeros(shape, dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    lse = torch.zeros((1, 2, 256), device="cuda")
+    acc = torch.zeros(shape, device="cuda")
+    bad = [
+        [(0, 0, 128, -1, 1, 1), (64, 0, 128, -1, 1, 1)],     # overlapping rows
+        [(200, 0, 128, -1, 1, 1)],                           # rows past the tensor
+        [(0, 200, 100, -1, 1, 1)],                           # keys past the tensor
+        [(0, 0, 0, -1, 1, 1)],                               # no keys
+        [(0, 0, 128, -1, 2, 1)],                             # a flag other than 0 / 1
+        [],                                                  # no segment
+        [(0, 0, 128, -1, 1, 1)] * 3,                         # three segments
+    ]
+    for segs in bad:
+        with pytest.raises(fa.FaError, match="INVALID_ARG"):
+            fa.ring_step(q, k, v, segs, 128, out, lse, acc=acc, layout="BSND")
+    with pytest.raises(fa.FaError, match="INVALID_ARG"):     # a running result is needed but missing
+        fa.ring_step(q, k, v, [(0, 0, 128, -1, 0, 1)], 128, out, lse, acc=None, layout="BSND")
+    big = torch.zeros(shape, device="cuda")                  # an fp32 acc whose first half is q
+    q_in_acc = big.view(torch.bfloat16).view(-1)[:q.numel()].view(shape)
+    with pytest.raises(fa.FaError, match="ALIAS"):
+        fa.ring_step(q_in_acc, k, v, [(0, 0, 128, -1, 1, 0)], 128, out, lse, acc=big, layout="BSND")
+    fa.check_device_status()
 
 
 RING_CASES = [
