@@ -978,15 +978,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (nt == 0) continue;
       const int row = un.r0 + t * BM + rit;          // query row of this thread
       const int first_row = un.r0 + t * BM;
+      // the rows the causal mask is taken at (a ring step's segment offsets them)
+      const int mrow = KIND == RING ? row + un.coff : row;
+      const int mfirst = KIND == RING ? first_row + un.coff : first_row;
+      const bool causal = KIND == RING ? (un.causal != 0) : (p.causal != 0);
       float m = -INFINITY;                           // running max, log2 domain
       float l = 0.f;                                 // running exp-sum (for the LSE)
       float ln = 0.f;                                // l with each tile's top weight as rounded in P (for O)
       float m_use = 0.f;
-      const int seg_flags = KIND == RING ? (un.seg ? p.seg_flags[1] : p.seg_flags[0]) : 0;
       for (int j = 0; j < nt; ++j) {
         if constexpr (KIND == RING) {
           // the running O row the epilogue merges with: into L2 while the last tile is computed
-          if (j + 1 == nt && !(seg_flags & 1) && row < un.sq) {
+          if (j + 1 == nt && !((un.seg ? p.seg_flags[1] : p.seg_flags[0]) & 1) && row < un.sq) {
             const float* a = p.acc + (size_t)un.b * p.o_bs + (size_t)un.h * p.o_hs + (size_t)(un.rb + row) * p.o_rs;
 #pragma unroll
             for (int i = 0; i < D / 32; ++i) prefetch_l2(a + 32 * i);
@@ -998,10 +1001,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++s_use;
         tc_fence_after();
         const int c0 = j * BN;
-        const bool masked = (c0 + BN > un.sk) || (un.causal && (c0 + BN - 1 > first_row + un.coff));
+        const bool masked = (c0 + BN > un.sk) || (causal && (c0 + BN - 1 > mfirst));
         const float cc = masked ? 1.f : c;
         int lim = un.sk - 1 - c0;
-        if (un.causal) lim = min(lim, row + un.coff - c0);
+        if (causal) lim = min(lim, mrow - c0);
         // this row of S_t from TMEM; diagonal / ragged tiles become scaled logits
         // with masked entries at -inf
         auto load_s = [&](uint32_t (&sr)[BN]) {
@@ -1092,28 +1095,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       ++o_use;
       tc_fence_after();
-      // Dense batch: O is staged (swizzled) in the Q tile's buffer and stored
-      // by TMA; the buffer is released once the store has read it.  Packed
-      // batch and ring step: each thread stores its own row from registers,
-      // and the MMA warp has already released the Q buffer after its last read.
       const bool store_row = row < un.sq;
-      const size_t lse_at = (size_t)un.b * p.lse_bs + (size_t)un.h * p.lse_hs + un.rb + row;
-      float lse2 = m_use + lg2(l);          // this result's LSE (log2 units)
-      float w_o = 1.f / ln;                 // O = w_o * O_tmem (+ w_run * running O)
-      float w_run = 0.f;
-      bool merge = false, final_o = true;
-      uint8_t* orow = nullptr;
-      float* arow = nullptr;
-      if constexpr (ROWSTORE) {
-        const size_t e = (size_t)un.b * p.o_bs + (size_t)un.h * p.o_hs + (size_t)(un.rb + row) * p.o_rs;
-        orow = p.o + e * 2;
-        if constexpr (KIND == RING) arow = p.acc + e;
-      }
       if constexpr (KIND == RING) {
-        // Merge with the running result (LSE a): the merged LSE is
+        // Ring step: merged with the running result of the rows (LSE a, fp32
+        // O in acc) unless this is their first result: the merged LSE is
         // log2(2^a + 2^lse2) and each part is weighted by 2^(its LSE - merged).
-        final_o = (seg_flags & 2) != 0;
-        merge = !(seg_flags & 1) && store_row;
+        // Stored as the running result (fp32) or, at the rows' last segment,
+        // as the output in the input dtype; each thread stores its own row.
+        const int seg_flags = un.seg ? p.seg_flags[1] : p.seg_flags[0];
+        const bool final_o = (seg_flags & 2) != 0;
+        const bool merge = !(seg_flags & 1) && store_row;
+        const size_t lse_at = (size_t)un.b * p.lse_bs + (size_t)un.h * p.lse_hs + un.rb + row;
+        const size_t e = (size_t)un.b * p.o_bs + (size_t)un.h * p.o_hs + (size_t)(un.rb + row) * p.o_rs;
+        uint8_t* orow = p.o + e * 2;
+        float* arow = p.acc + e;
+        float lse2 = m_use + lg2(l);          // this segment's LSE (log2 units)
+        float w_o = 1.f / ln, w_run = 0.f;    // O = w_o * O_tmem + w_run * running O
         if (merge) {
           const float a = p.lse[lse_at] * 1.44269504088896340736f;
           const float mx = fmaxf(a, lse2);
@@ -1123,75 +1120,102 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           w_o *= eb * inv;
           lse2 = mx + lg2(ea + eb);
         }
-      }
-      {
         uint32_t r[32];
-        float4 run[8];     // 32 columns of the running O row
-        // (a ring step keeps this loop rolled: unrolled, the running O loads
-        // of every chunk are hoisted together and the registers spill)
-#pragma unroll(KIND == RING ? 1 : D / 32)
+        // (kept rolled: unrolled, the running O loads of every chunk are
+        // hoisted together and the registers spill)
+#pragma unroll 1
         for (int q4 = 0; q4 < D / 32; ++q4) {
-          if constexpr (KIND == RING) {
-            if (merge) {
-              const float4* src = reinterpret_cast<const float4*>(arow) + q4 * 8;
-#pragma unroll
-              for (int i = 0; i < 8; ++i) run[i] = src[i];
-            }
-          }
           tmem_ld32(tO + q4 * 32, r);
           tmem_wait_ld();
           reg_fence(r);
-          float f[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(r[i]) * w_o;
-          if constexpr (KIND == RING) {
-            if (merge) {
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * w_o);
+          if (merge) {
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                f[4 * i] += run[i].x * w_run;
-                f[4 * i + 1] += run[i].y * w_run;
-                f[4 * i + 2] += run[i].z * w_run;
-                f[4 * i + 3] += run[i].w * w_run;
+            for (int h = 0; h < 2; ++h) {
+              const float4* src = reinterpret_cast<const float4*>(arow) + q4 * 8 + h * 4;
+              float4 run[4];     // 16 columns of the running O row
+#pragma unroll
+              for (int i = 0; i < 4; ++i) run[i] = src[i];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                uint32_t* x = &r[16 * h + 4 * i];
+                x[0] = __float_as_uint(fmaf(run[i].x, w_run, __uint_as_float(x[0])));
+                x[1] = __float_as_uint(fmaf(run[i].y, w_run, __uint_as_float(x[1])));
+                x[2] = __float_as_uint(fmaf(run[i].z, w_run, __uint_as_float(x[2])));
+                x[3] = __float_as_uint(fmaf(run[i].w, w_run, __uint_as_float(x[3])));
               }
-            }
-            if (!final_o) {
-              if (store_row) {
-                float4* dst = reinterpret_cast<float4*>(arow) + q4 * 8;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) dst[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
-              }
-              continue;
             }
           }
-          uint32_t w[16];
+          if (!store_row) continue;
+          if (final_o) {
+            uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(f[2 * i], f[2 * i + 1]);
-          if constexpr (ROWSTORE) {
-            if (store_row) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 64);
+            for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 64);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-            }
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
           } else {
-            // row rit of box q4/2, 16-byte chunks (q4&1)*4 + i, 128-byte swizzle
-            uint8_t* rowp = sQt + (q4 >> 1) * BOX_BYTES + rit * 128;
+            uint4* dst = reinterpret_cast<uint4*>(arow) + q4 * 8;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int chunk = ((q4 & 1) * 4 + i) ^ (rit & 7);
-              *reinterpret_cast<uint4*>(rowp + chunk * 16) =
-                  make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            for (int i = 0; i < 8; ++i) dst[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+          }
+        }
+        if (store_row) p.lse[lse_at] = lse2 * 0.69314718055994530942f;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::O_EMPTY + t));
+      } else {
+        const float inv_l = 1.f / ln;
+        // Dense batch: O is staged (swizzled) in the Q tile's buffer and
+        // stored by TMA; the buffer is released once the store has read it.
+        // Packed (variable-length) batch: each thread stores its own row
+        // from registers -- a tile may end inside the sequence, where a TMA
+        // store would also write the next sequence's rows -- and the MMA warp
+        // has already released the Q buffer after its last read.
+        uint8_t* orow = nullptr;
+        if constexpr (KIND == PACKED) orow = p.o + ((size_t)(un.rb + row) * p.H + un.h) * (D * 2);
+        {
+          uint32_t r[32];
+#pragma unroll
+          for (int q4 = 0; q4 < D / 32; ++q4) {
+            tmem_ld32(tO + q4 * 32, r);
+            tmem_wait_ld();
+            reg_fence(r);
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
+            if constexpr (KIND == PACKED) {
+              if (store_row) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 64);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+              }
+            } else {
+              // row rit of box q4/2, 16-byte chunks (q4&1)*4 + i, 128-byte swizzle
+              uint8_t* rowp = sQt + (q4 >> 1) * BOX_BYTES + rit * 128;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int chunk = ((q4 & 1) * 4 + i) ^ (rit & 7);
+                *reinterpret_cast<uint4*>(rowp + chunk * 16) =
+                    make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+              }
             }
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::O_EMPTY + t));
+        if constexpr (!ROWSTORE) {
+          fence_proxy_async_smem();
+          mbar_arrive(bar(C::EPI + t));
+        }
+        if (store_row) {
+          const float lse = (m_use + lg2(l)) * 0.69314718055994530942f;
+          p.lse[(size_t)un.b * p.lse_bs + (size_t)un.h * p.lse_hs + un.rb + row] = lse;
+        }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::O_EMPTY + t));
-      if constexpr (!ROWSTORE) {
-        fence_proxy_async_smem();
-        mbar_arrive(bar(C::EPI + t));
-      }
-      if (store_row) p.lse[lse_at] = lse2 * 0.69314718055994530942f;
       if constexpr (!ROWSTORE) {
         if (rit == 0) {
           // one thread stores the tile once all 128 rows are staged
