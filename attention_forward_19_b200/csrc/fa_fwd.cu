@@ -494,26 +494,32 @@ __device__ __forceinline__ uint32_t imad_shl23(uint32_t a, uint32_t b) {
   return d;
 }
 
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // 2^x for two values on the FMA pipe instead of MUFU.  x = j + r with
 // j = round(x): adding 1.5 * 2^23 leaves j in the low mantissa bits, so
-// 1.5 * 2^23 - (x + 1.5 * 2^23) = -j exactly and r = x - j lies in [-1/2, 1/2].
+// (x + 1.5 * 2^23) - 1.5 * 2^23 = j exactly and r = x - j lies in [-1/2, 1/2].
 // 2^r is a polynomial (constant term 1; near-minimax in relative error, fitted
 // by csrc/gen_exp2_poly.py: 1.0e-4 at degree 3, 2.9e-6 at degree 4), and 2^j
-// is added to its exponent field.  x is clamped to [-125, 64] so the exponent
-// stays normal: 2^-125 stands in for any finite value below (-inf, a masked
-// key, gives exactly 0), and an argument above 64 (only possible on a
-// rejected speculative pass, see the softmax) still gives a large positive
-// value.
+// is added to its exponent field.  x is clamped to [-127, 64]: at -127, r = 0
+// and the polynomial is exactly 1, whose exponent field 127 the addition
+// takes to zero, so -inf (a masked key) and anything below give exactly +0;
+// just above -127 the result is a denormal below 2^-126 (negligible beside
+// the row's largest weight, at least 2^-headroom); an argument above 64
+// (only possible on a rejected speculative pass, see the softmax) still gives
+// a large positive value.
 template <int DEG>
 __device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& y0, float& y1) {
   float xin0, xin1;
   f2unpack(x2, xin0, xin1);
-  const float x0 = fminf(fmaxf(xin0, -125.f), 64.f);
-  const float x1 = fminf(fmaxf(xin1, -125.f), 64.f);
+  const uint64_t x = f2pack(fminf(fmaxf(xin0, -127.f), 64.f), fminf(fmaxf(xin1, -127.f), 64.f));
   const uint64_t magic = f2pack(12582912.f, 12582912.f);
-  const uint64_t t = fadd2(f2pack(x0, x1), magic);
-  const uint64_t neg_j = ffma2(t, f2pack(-1.f, -1.f), magic);
-  const uint64_t r = fadd2(f2pack(x0, x1), neg_j);
+  const uint64_t t = fadd2(x, magic);
+  const uint64_t r = fsub2(x, fsub2(t, magic));
   uint64_t p;
   if constexpr (DEG == 3) {
     p = ffma2(r, f2pack(5.500874668e-02f, 5.500874668e-02f), f2pack(2.422107607e-01f, 2.422107607e-01f));
@@ -531,9 +537,6 @@ __device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& y0, float& y1
   // which runs on the FMA pipe); bits(t) * 2^23 keeps only j * 2^23 modulo 2^32
   y0 = __uint_as_float(imad_shl23(__float_as_uint(t0), __float_as_uint(p0)));
   y1 = __uint_as_float(imad_shl23(__float_as_uint(t1), __float_as_uint(p1)));
-  // a masked key (-inf) weighs exactly 0, as MUFU's ex2 gives
-  y0 = xin0 >= -125.f ? y0 : 0.f;
-  y1 = xin1 >= -125.f ? y1 : 0.f;
 }
 
 // max over the row of s * c (c > 0: max(s) * c; c < 0: min(s) * c; c = 0: 0).
