@@ -389,7 +389,9 @@ def run_native(args, rank, world, local_rank):
     if os.path.exists(TRAFFIC_FILE):
         with open(TRAFFIC_FILE) as f:
             tr = json.load(f)
-        if tr.get("kernel_sha256_16") == kernel_hash():
+        if tr.get("workload") != w0.name:
+            traffic_note = f"the ncu traffic capture is of {tr.get('workload')}, not this workload"
+        elif tr.get("kernel_sha256_16") == kernel_hash():
             traffic = tr.get("dram_bytes_per_launch")
             traffic_note = tr.get("note", "")
         else:
