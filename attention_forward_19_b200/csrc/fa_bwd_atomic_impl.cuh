@@ -22,7 +22,9 @@
 // global memory with red.global.add.f32 from registers: one warp instruction
 // covers 128 contiguous bytes of a query row.  (Staging the tile in shared
 // memory for one 32 KB bulk reduction was 12 % slower: two more barriers, a
-// proxy fence and one thread issuing.)  A last kernel scales the accumulator
+// proxy fence and one thread issuing.)  The adds are made by a warpgroup of
+// their own (warps 12-15, one per TMEM lane quadrant), so that the compute
+// warps go on to the next step's P^T while a step's dQ is added.  A last kernel scales the accumulator
 // and rounds it into dq.  The 64-query step keeps the TMEM budget at 512
 // columns; the stream of Q / dO sub-tiles has three stages.
 // D = 64: dQ^T = K^T dS^T is still an M = 128 product (the layout the other
@@ -35,7 +37,14 @@ namespace bwda {
 
 using bwd::LOAD_WARP;
 using bwd::MMA_WARP;
-using bwd::THREADS;
+// 16 warps: 0-7 compute, 8 load, 9 MMA, 10-11 idle, 12-15 dQ adders.  The
+// launch gives 512 x 128 registers; setmaxnreg raises the compute warpgroups
+// to 168 and lowers the other two to 88: 256 x 168 + 256 x 88 = 65536.
+constexpr int THREADS_A = 512;
+constexpr int ADD_WARP0 = 12;
+constexpr int REGS_COMPUTE = 168;
+constexpr int REGS_OTHER = 88;
+static_assert(256 * REGS_COMPUTE + 256 * REGS_OTHER <= 65536, "register split exceeds the launch");
 
 constexpr int SUB = 64;          // queries per step
 constexpr int NST = 3;           // streamed stages (a Q and a dO sub-tile, two vectors)
@@ -104,7 +113,7 @@ __device__ __forceinline__ void load_sub(uint32_t dst, const CUtensorMap* map, u
 }
 
 template <int DH, bool BF16>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS_A, 1)
     dkdvq_kernel(const __grid_constant__ bwd::Params p, const __grid_constant__ CUtensorMap tmQ64,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const __grid_constant__ CUtensorMap tmDO64) {
@@ -143,7 +152,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(bar(DP_FULL), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(DQ_FULL + i), 1);
-      mbar_init(bar(RD_C + i), 2 * BM);
+      mbar_init(bar(RD_C + i), 4);      // one arrival per adder warp
     }
     mbar_init(bar(W_A), 2 * BM);
     mbar_init(bar(W_B), 2 * BM);
@@ -173,7 +182,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   constexpr uint32_t IDESC_ACC = idesc_ab(BM, DH, FMT, 0, 1);    // 128 keys x D, A in TMEM, B MN-major
   constexpr uint32_t IDESC_DQ = idesc_ab(BM, SUB, FMT, 1, 1);    // 128 (D, zero-padded) x 64 queries, MN-major
 
-  if (warp == LOAD_WARP) {
+  if (warp >= LOAD_WARP && warp < ADD_WARP0) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
+   if (warp == LOAD_WARP) {
     if (lane == 0 && nu > 0) {
       bool ok = true;
       mbar_arrive_expect_tx(bar(IN_FULL), 2 * A::VT_BYTES);
@@ -199,7 +210,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (uint32_t c = first; c < issued; ++c) drain_wait(bar(ST_FULL + c % NST), (c / NST) & 1u, limit);
     }
     __syncwarp();
-  } else if (warp == MMA_WARP) {
+   } else if (warp == MMA_WARP) {
     if (nu > 0) {
       bool ok = wait_bar(bar(IN_FULL), 0, abort_flag, limit);
       const uint64_t dKk = sdesc(sFix, 16, 1024), dVk = sdesc(sFix + A::SMEM_V, 16, 1024);
@@ -289,9 +300,43 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) drain_wait(bar(DRAIN), 0, limit);
     }
     __syncwarp();
+   }
+  } else if (warp >= ADD_WARP0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_OTHER));
+    // ---------------------------------------------------------------- dQ adders: lane = head-dim index
+    // Warp 12 + q reads TMEM lane quadrant (12 + q) % 4 = q of each dQ_v^T tile
+    // (head-dim rows, 64 query columns) and adds it to the fp32 accumulator:
+    // one warp instruction covers 128 contiguous bytes of one query row.  At
+    // D = 64 the lanes 64-127 (zero rows) are read but not added.
+    const int quad = warp & 3;
+    const int drow = quad * 32 + lane;
+    const uint32_t lane_bits = (uint32_t)(quad * 32) << 16;
+    float* dq_acc_bh = p.dq_acc + (size_t)bh * p.Sq_pad * DH;
+    for (uint32_t v = 0; v < (uint32_t)nu; ++v) {
+      if (!wait_bar(bar(DQ_FULL + (v & 1u)), (v >> 1) & 1u, abort_flag, limit)) break;
+      tc_fence_after();
+      uint32_t r[2][32];
+      tmem_ld32(tmem + lane_bits + COL_DQ + (v & 1u) * SUB, r[0]);
+      tmem_ld32(tmem + lane_bits + COL_DQ + (v & 1u) * SUB + 32, r[1]);
+      tmem_wait_ld();
+      reg_fence(r[0]);
+      reg_fence(r[1]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(RD_C + (v & 1u)));
+      if (drow < DH) {
+        float* dst = dq_acc_bh + (size_t)(u_begin + (int)v) * SUB * DH + drow;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) atomicAdd(dst + (size_t)(32 * h + j) * DH, __uint_as_float(r[h][j]));
+      }
+    }
+    __syncwarp();
   } else {
-    // ---------------------------------------------------------------- compute: one thread per key (phases A, B),
-    // one per head-dim index (phase C); group g takes queries [32 g, 32 g + 32) of a step
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_COMPUTE));
+    // ---------------------------------------------------------------- compute: one thread per key (phases A, B);
+    // group g takes queries [32 g, 32 g + 32) of a step
     const int quad = warp & 3, grp = warp >> 2;
     const int rit = quad * 32 + lane;
     const int key = k0 + rit;
@@ -300,27 +345,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tST = tmem + lane_bits + COL_ST, tDPT = tmem + lane_bits + COL_DPT;
     const uint32_t tDV = tmem + lane_bits + COL_DV, tDK = tmem + lane_bits + COL_DK;
     const float c = p.scale_log2;
-    float* dq_acc_bh = p.dq_acc + (size_t)bh * p.Sq_pad * DH;
     bool ok = true;
-    // phase C of step v: thread rit adds column rit of dQ_v (its 32 queries) to the
-    // accumulator; a warp's add covers 128 contiguous bytes of one query row.  At
-    // D = 64 the TMEM lanes 64-127 (zero rows) are read but not added.
-    auto phase_c = [&](uint32_t v) -> bool {
-      if (!wait_bar(bar(DQ_FULL + (v & 1u)), (v >> 1) & 1u, abort_flag, limit)) return false;
-      tc_fence_after();
-      uint32_t r[32];
-      tmem_ld32(tmem + lane_bits + COL_DQ + (v & 1u) * SUB + grp * 32, r);
-      tmem_wait_ld();
-      reg_fence(r);
-      tc_fence_before();
-      mbar_arrive(bar(RD_C + (v & 1u)));
-      if (rit < DH) {
-        float* dst = dq_acc_bh + ((size_t)(u_begin + (int)v) * SUB + grp * 32) * DH + rit;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) atomicAdd(dst + (size_t)j * DH, __uint_as_float(r[j]));
-      }
-      return true;
-    };
     for (uint32_t u = 0; u < (uint32_t)nu && ok; ++u) {
       const uint32_t st = u % NST;
       ok = wait_bar(bar(ST_FULL + st), (u / NST) & 1u, abort_flag, limit);   // the vectors came by bulk copy
@@ -394,13 +419,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(W_B));
-      // ---- phase C of the previous step
-      if (u >= 1) {
-        ok = phase_c(u - 1);
-        if (!ok) break;
-      }
     }
-    if (ok && nu > 0) ok = phase_c((uint32_t)nu - 1);
     // ---------------------------------------------------------------- epilogue: dV and scale * dK rows
     const bool store = key < p.Sk;
     uint8_t* dvrow = p.dv + (size_t)b * p.k_bs + (size_t)h * p.k_hs + (size_t)key * p.k_rs;
@@ -495,7 +514,7 @@ fa_status launch_bwd_atomic(fa::bwd::Params& prm, const CUtensorMap& mq64, const
   if (e != cudaSuccess) return cuda_fail((int)e);
   e = cudaMemsetAsync(prm.dq_acc, 0, (size_t)rows * DH * sizeof(float), s);
   if (e != cudaSuccess) return cuda_fail((int)e);
-  kern<<<(unsigned)(prm.B * prm.H * prm.tk), fa::bwd::THREADS, smem, s>>>(prm, mq64, mk, mv, mdo64);
+  kern<<<(unsigned)(prm.B * prm.H * prm.tk), fa::bwda::THREADS_A, smem, s>>>(prm, mq64, mk, mv, mdo64);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail((int)e);
   const long long qrows = (long long)prm.B * prm.H * prm.Sq;
