@@ -17,15 +17,14 @@
 //                                           K^T is the K tile read MN-major, dS^T
 //                                           is written there by the compute warps)
 // TMEM: dV [0,128) | dK [128,256) | S^T [256,320) | dP^T [320,384) |
-// dQ^T [384,448) and [448,512) (two buffers).  The compute warps read each
-// dQ_u^T tile (lanes = head-dim index) and add it to the fp32 accumulator in
-// global memory with red.global.add.f32 from registers: one warp instruction
-// covers 128 contiguous bytes of a query row.  (Staging the tile in shared
-// memory for one 32 KB bulk reduction was 12 % slower: two more barriers, a
-// proxy fence and one thread issuing.)  The adds are made by a warpgroup of
-// their own (warps 12-15, one per TMEM lane quadrant), so that the compute
-// warps go on to the next step's P^T while a step's dQ is added.  A last kernel scales the accumulator
-// and rounds it into dq.  The 64-query step keeps the TMEM budget at 512
+// dQ^T [384,448) and [448,512) (two buffers).  A warpgroup of its own
+// (warps 12-15, one per TMEM lane quadrant) reads each dQ_u^T tile (lanes =
+// head-dim index) and adds it to the fp32 accumulator in global memory with
+// red.global.add.f32 from registers, one warp instruction per 128 contiguous
+// bytes of a query row, while the compute warps go on to the next step's P^T.
+// (Staging the tile in shared memory for one 32 KB bulk reduction was 12 %
+// slower: two more barriers, a proxy fence and one thread issuing.)  A last
+// kernel scales the accumulator and rounds it into dq.  The 64-query step keeps the TMEM budget at 512
 // columns; the stream of Q / dO sub-tiles has three stages.
 // D = 64: dQ^T = K^T dS^T is still an M = 128 product (the layout the other
 // products use): the K tile's region holds two 64-column boxes as at D = 128,
