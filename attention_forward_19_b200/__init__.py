@@ -40,7 +40,8 @@ LAYOUTS = {"BSND": FA_BSND, "BHSD": FA_BHSD}
 
 # Names every public symbol of include/fa_fwd.h.
 EXPORTED_SYMBOLS = ("fa_fwd", "fa_fwd_ws", "fa_fwd_workspace_size", "fa_fwd_opts", "fa_fwd_default_options",
-                    "fa_fwd_heads", "fa_fwd_noalloc", "fa_fwd_varlen",
+                    "fa_fwd_heads", "fa_fwd_noalloc", "fa_fwd_varlen", "fa_fwd_splitkv",
+                    "fa_fwd_splitkv_workspace_size",
                     "fa_bwd",
                     "fa_bwd_workspace_size", "fa_bwd_atomic",
                     "fa_bwd_atomic_workspace_size", "fa_lse_merge", "fa_fwd_ring_step", "fa_out_proj",
@@ -119,6 +120,11 @@ def load_library(path=None, rebuild_if_stale=True):
                            vp, ctypes.c_size_t, vp]
     lib.fa_lse_merge.restype = c_int
     lib.fa_lse_merge.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, c_int, c_int, c_int, vp]
+    lib.fa_fwd_splitkv.restype = c_int
+    lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, c_int, c_float, c_int, c_int, vp,
+                                   ctypes.c_size_t, vp]
+    lib.fa_fwd_splitkv_workspace_size.restype = ctypes.c_size_t
+    lib.fa_fwd_splitkv_workspace_size.argtypes = [i64, i64, i64, i64, c_int]
     lib.fa_fwd_ring_step.restype = c_int
     lib.fa_fwd_ring_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.POINTER(RingSegment),
                                      c_int, c_int, c_float, c_int, vp, ctypes.c_size_t, vp]
@@ -226,6 +232,18 @@ def fa_lse_merge(o_part, lse_part, o_acc, lse_acc, o_out, lse_out, B, H, S, D, l
     lib = load_library()
     return lib.fa_lse_merge(o_part, lse_part, o_acc, lse_acc, o_out, lse_out, int(B), int(H), int(S), int(D),
                             int(layout), int(dtype), int(flags), stream)
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, B, H, Sq, Sk, D, layout, scale, dtype, nsplit, workspace, workspace_bytes,
+                   stream):
+    """The C fa_fwd_splitkv with raw pointers and sizes; returns the fa_status code."""
+    lib = load_library()
+    return lib.fa_fwd_splitkv(q, k, v, o, lse, int(B), int(H), int(Sq), int(Sk), int(D), int(layout), float(scale),
+                              int(dtype), int(nsplit), workspace, int(workspace_bytes), stream)
+
+
+def fa_fwd_splitkv_workspace_size(B, H, Sq, D, nsplit):
+    return load_library().fa_fwd_splitkv_workspace_size(int(B), int(H), int(Sq), int(D), int(nsplit))
 
 
 def fa_fwd_ring_step(q, k, v, o, acc, lse, B, H, Sq, Sk, D, rows, segs, layout, scale, dtype, workspace,
@@ -605,6 +623,45 @@ def lse_merge(o_part, lse_part, o_acc=None, lse_acc=None, out=None, lse_out=None
     if st != FA_OK:
         raise FaError(st, "fa_lse_merge")
     return (out, lse_out) if final else (o_acc, lse_acc)
+
+
+def default_splits(B, H, Sq, Sk, sms=148):
+    """A split count for flash_attention_forward_splitkv: enough key ranges to give every SM about one
+    work unit (units of 256 query rows), each range at least 8 key tiles of 128 (a shorter range does not
+    pay for the merge kernel: at 512 keys, c1, one pass takes 14.6 us and two ranges 17.9 us), at most
+    64; 1 means the one-pass kernel is the better choice."""
+    units = B * H * ((Sq + 255) // 256)
+    return max(1, min(64, ((Sk + 127) // 128) // 8, sms // max(1, units)))
+
+
+def flash_attention_forward_splitkv(q, k, v, layout="BSND", scale=None, nsplit=None, out=None, lse=None,
+                                    workspace=None, stream=None):
+    """Attention without a mask through fa_fwd_splitkv: the key range split into nsplit ranges (default
+    default_splits(...)), each a work unit of its own, the partial results merged by a second kernel.
+    Arguments and results as for flash_attention_forward (causal=False)."""
+    import torch
+    lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    B, H, Sq, Sk, D = _dims(q, k, lay)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if nsplit is None:
+        nsplit = default_splits(B, H, Sq, Sk, torch.cuda.get_device_properties(q.device).multi_processor_count)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device) if lse is None else lse
+    need = fa_fwd_splitkv_workspace_size(B, H, Sq, D, nsplit)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    sptr = stream.cuda_stream if hasattr(stream, "cuda_stream") else stream
+    st = fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Sq, Sk, D,
+                        lay, scale, _dtype_code(q), nsplit, workspace.data_ptr(), workspace.numel(), sptr)
+    if st != FA_OK:
+        raise FaError(st, "fa_fwd_splitkv")
+    return out, lse
 
 
 def ring_step(q, k, v, segments, rows, out, lse, acc=None, layout="BSND", scale=None, workspace=None, stream=None):

@@ -150,6 +150,12 @@ struct Params {
   int nseg, seg_units0;
   int seg_row0[2], seg_key0[2], seg_sk[2], seg_coff[2], seg_causal[2], seg_flags[2];
   float* acc;
+  // Split-KV (a ring-step launch with split_n > 0 instead of segments): split
+  // s takes keys [s * split_keys, (s + 1) * split_keys) of every query row
+  // (no mask) and writes its own result as the rows' first, not last, one:
+  // fp32 O to rows s * Sq + r of acc and its LSE to the same rows of lse;
+  // units of split s are [s * seg_units0, (s + 1) * seg_units0).
+  int split_n, split_keys;
   // Lazy rescale: the reference max moves only when a tile's max exceeds it
   // by more than rescale_log2 (weights against a stale reference stay below
   // rescale_pow2 = 2^rescale_log2); bf16 sets a moved reference headroom_log2
@@ -619,7 +625,8 @@ constexpr int DENSE = 0, PACKED = 1, RING = 2;
 struct Unit {
   int b, h, r0;     // batch, head, first query row of the unit (within its sequence)
   int causal, coff; // causal mask (key c visible from row r iff c <= r + coff)
-  int seg;          // ring-step segment
+  int seg;          // ring-step segment (or split)
+  int ob;           // first row of the unit's results in O / LSE (ring step and split-KV)
   int rows[NQ];     // valid rows of each query tile
   int n[NQ];        // key tiles each query tile visits (0: tile inactive)
   int sq, sk;       // the sequence's query and key lengths
@@ -638,10 +645,16 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
   if constexpr (KIND == RING) {
     // (selects rather than indexing: a dynamic index into the parameters
     // would copy them to local memory)
-    un.seg = u >= p.seg_units0 ? 1 : 0;
-    if (un.seg) u -= p.seg_units0;
-    un.causal = un.seg ? p.seg_causal[1] : p.seg_causal[0];
-    un.coff = un.seg ? p.seg_coff[1] : p.seg_coff[0];
+    if (p.split_n > 0) {
+      un.seg = u / p.seg_units0;
+      u -= un.seg * p.seg_units0;
+      un.causal = 0;
+    } else {
+      un.seg = u >= p.seg_units0 ? 1 : 0;
+      if (un.seg) u -= p.seg_units0;
+      un.causal = un.seg ? p.seg_causal[1] : p.seg_causal[0];
+      un.coff = un.seg ? p.seg_coff[1] : p.seg_coff[0];
+    }
   }
   const int per_group = p.group_heads * p.nqb;
   const int g = u / per_group;
@@ -666,18 +679,28 @@ __device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
     un.rb = q0;
     un.kb = k0;
     un.tb = 0;
+    un.ob = q0;
   } else if constexpr (KIND == RING) {
     un.sq = p.Sq;
-    un.sk = un.seg ? p.seg_sk[1] : p.seg_sk[0];
-    un.rb = un.seg ? p.seg_row0[1] : p.seg_row0[0];
-    un.kb = un.seg ? p.seg_key0[1] : p.seg_key0[0];
     un.tb = un.b;
+    if (p.split_n > 0) {
+      un.kb = un.seg * p.split_keys;
+      un.sk = min(p.split_keys, p.Sk - un.kb);
+      un.rb = 0;
+      un.ob = un.seg * p.Sq;
+    } else {
+      un.sk = un.seg ? p.seg_sk[1] : p.seg_sk[0];
+      un.rb = un.seg ? p.seg_row0[1] : p.seg_row0[0];
+      un.kb = un.seg ? p.seg_key0[1] : p.seg_key0[0];
+      un.ob = un.rb;
+    }
   } else {
     un.sq = p.Sq;
     un.sk = p.Sk;
     un.rb = 0;
     un.kb = 0;
     un.tb = un.b;
+    un.ob = 0;
   }
 #pragma unroll
   for (int t = 0; t < NQ; ++t) {
@@ -992,8 +1015,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int j = 0; j < nt; ++j) {
         if constexpr (KIND == RING) {
           // the running O row the epilogue merges with: into L2 while the last tile is computed
-          if (j + 1 == nt && !((un.seg ? p.seg_flags[1] : p.seg_flags[0]) & 1) && row < un.sq) {
-            const float* a = p.acc + (size_t)un.b * p.o_bs + (size_t)un.h * p.o_hs + (size_t)(un.rb + row) * p.o_rs;
+          if (j + 1 == nt && p.split_n == 0 && !((un.seg ? p.seg_flags[1] : p.seg_flags[0]) & 1) && row < un.sq) {
+            const float* a = p.acc + (size_t)un.b * p.o_bs + (size_t)un.h * p.o_hs + (size_t)(un.ob + row) * p.o_rs;
 #pragma unroll
             for (int i = 0; i < D / 32; ++i) prefetch_l2(a + 32 * i);
           }
@@ -1105,11 +1128,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // log2(2^a + 2^lse2) and each part is weighted by 2^(its LSE - merged).
         // Stored as the running result (fp32) or, at the rows' last segment,
         // as the output in the input dtype; each thread stores its own row.
-        const int seg_flags = un.seg ? p.seg_flags[1] : p.seg_flags[0];
+        // (a split-KV split is always its rows' first result and never their last)
+        const int seg_flags = p.split_n > 0 ? 1 : (un.seg ? p.seg_flags[1] : p.seg_flags[0]);
         const bool final_o = (seg_flags & 2) != 0;
         const bool merge = !(seg_flags & 1) && store_row;
-        const size_t lse_at = (size_t)un.b * p.lse_bs + (size_t)un.h * p.lse_hs + un.rb + row;
-        const size_t e = (size_t)un.b * p.o_bs + (size_t)un.h * p.o_hs + (size_t)(un.rb + row) * p.o_rs;
+        const size_t lse_at = (size_t)un.b * p.lse_bs + (size_t)un.h * p.lse_hs + un.ob + row;
+        const size_t e = (size_t)un.b * p.o_bs + (size_t)un.h * p.o_hs + (size_t)(un.ob + row) * p.o_rs;
         uint8_t* orow = p.o + e * 2;
         float* arow = p.acc + e;
         float lse2 = m_use + lg2(l);          // this segment's LSE (log2 units)

@@ -107,6 +107,68 @@ __global__ void __launch_bounds__(THREADS) merge_kernel(const __grid_constant__ 
   }
 }
 
+// Split-KV: a row's nsplit partial results, each normalised over its own key
+// range (fp32 O at row s * S + r of a [B * H, nsplit * S, D] buffer, its LSE
+// at the same row of [B * H, nsplit * S]), merged in one pass by the same
+// update taken over all of them at once:
+//   LSE = M + log(sum_s exp(LSE_s - M)),  O = sum_s exp(LSE_s - LSE) O_s,
+// with M the largest LSE_s (a split with LSE_s = -inf has weight 0).  One warp
+// per row, D / 32 columns per lane; O is written in the 16-bit input type in
+// the caller's layout, LSE as fp32 [B, H, S].
+template <int D, bool BF16>
+__global__ void __launch_bounds__(THREADS) splitkv_merge_kernel(const float* __restrict__ o_part,
+                                                                const float* __restrict__ lse_part, uint16_t* o,
+                                                                float* lse, long long rows, int H, int S, int nsplit,
+                                                                int bhsd) {
+  constexpr int PER = D / 32;
+  constexpr float LOG2E = 1.44269504088896340736f;
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * (THREADS / 32) + (threadIdx.x >> 5);   // [B, H, S] order
+  if (row >= rows) return;
+  const long long bh = row / S;
+  const int r = (int)(row - bh * S);
+  const size_t base = (size_t)bh * nsplit * S + r;
+  float m = -INFINITY;
+  for (int s = lane; s < nsplit; s += 32) m = fmaxf(m, lse_part[base + (size_t)s * S]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  float acc[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  float wsum = 0.f;
+  if (m > -INFINITY) {
+    for (int s = 0; s < nsplit; ++s) {
+      const float ls = lse_part[base + (size_t)s * S];
+      if (!(ls > -INFINITY)) continue;
+      const float w = ex2((ls - m) * LOG2E);
+      wsum += w;
+      const float* src = o_part + (base + (size_t)s * S) * D + lane * PER;
+      if constexpr (PER == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src);
+        acc[0] += w * x.x;
+        acc[1] += w * x.y;
+        acc[2] += w * x.z;
+        acc[3] += w * x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(src);
+        acc[0] += w * x.x;
+        acc[1] += w * x.y;
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  const long long b = bh / H, h = bh - b * H;
+  const size_t orow = bhsd ? (size_t)(bh * S + r) : (size_t)((b * S + r) * H + h);
+  uint16_t* dst = o + orow * D + lane * PER;
+  uint32_t w2[PER / 2];
+#pragma unroll
+  for (int i = 0; i < PER / 2; ++i)
+    w2[i] = (uint32_t)from_f32(acc[2 * i] * inv, BF16) | ((uint32_t)from_f32(acc[2 * i + 1] * inv, BF16) << 16);
+  if constexpr (PER == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(w2[0], w2[1]);
+  else *reinterpret_cast<uint32_t*>(dst) = w2[0];
+  if (lane == 0) lse[row] = m > -INFINITY ? m + lg2(wsum) * 0.69314718055994530942f : -INFINITY;
+}
+
 }  // namespace merge
 }  // namespace fa
 
@@ -192,6 +254,110 @@ fa_status fa_lse_merge(const void* o_part, const float* lse_part, float* o_acc, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return dtype == FA_BF16 ? launch_merge<true>(prm, has_acc, final_, grid, s)
                           : launch_merge<false>(prm, has_acc, final_, grid, s);
+}
+
+// Workspace of fa_fwd_splitkv: the work counter (256 bytes kept for it), the
+// partial LSEs and the partial O rows, all for nsplit splits.
+static size_t splitkv_ws_bytes(int64_t B, int64_t H, int64_t Sq, int64_t D, int64_t nsplit) {
+  const size_t rows = (size_t)(B * H * nsplit * Sq);
+  return 256 + ((rows * 4 + 15) & ~(size_t)15) + rows * (size_t)D * 4;
+}
+
+size_t fa_fwd_splitkv_workspace_size(int64_t B, int64_t H, int64_t Sq, int64_t D, int nsplit) {
+  if (B <= 0 || H <= 0 || Sq < 0 || (D != 64 && D != 128) || nsplit < 1 || nsplit > 64) return 0;
+  return splitkv_ws_bytes(B, H, Sq, D, nsplit);
+}
+
+fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                         int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, float scale, fa_dtype dtype, int nsplit,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  bool noop = false;
+  fa_status hst = host_checks(q, k, v, o, lse, B, H, Sq, Sk, D, layout, scale, dtype, &noop);
+  if (hst != FA_OK) return hst;
+  if (nsplit < 1 || nsplit > 64) return FA_ERR_INVALID_ARG;
+  if (noop) return FA_OK;
+  // splits of whole key tiles: split_keys keys each (the last may be shorter)
+  const int64_t per = (Sk + nsplit - 1) / nsplit;
+  const int64_t split_keys = (per + fa::BN - 1) / fa::BN * fa::BN;
+  const int64_t n_eff = (Sk + split_keys - 1) / split_keys;
+  const size_t need = splitkv_ws_bytes(B, H, Sq, D, n_eff);
+  if (!workspace || workspace_bytes < splitkv_ws_bytes(B, H, Sq, D, nsplit) || workspace_bytes < need)
+    return FA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_MISALIGNED;
+  const int64_t nqb = (Sq + fa::UNIT_ROWS - 1) / fa::UNIT_ROWS;
+  if (n_eff * B * H * nqb >= ((int64_t)1 << 30) || B * H * n_eff * Sq >= ((int64_t)1 << 31)) return FA_ERR_UNSUPPORTED;
+  {
+    const size_t qbytes = (size_t)(B * H * Sq * D) * 2, kvbytes = (size_t)(B * H * Sk * D) * 2;
+    const size_t lbytes = (size_t)(B * H * Sq) * 4;
+    const void* bufs[5] = {q, k, v, o, lse};
+    const size_t sizes[5] = {qbytes, kvbytes, kvbytes, qbytes, lbytes};
+    for (int j = 0; j < 5; ++j)
+      if (overlaps(workspace, workspace_bytes, bufs[j], sizes[j])) return FA_ERR_ALIAS;
+  }
+  int dev = 0, sms = 0;
+  const void* ptrs[6] = {q, k, v, o, lse, workspace};
+  fa_status st = device_checks(ptrs, 6, &dev, &sms);
+  if (st != FA_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map(&mq, q, dtype, layout, B, H, Sq, D)) != FA_OK) return st;
+  if ((st = make_map(&mk, k, dtype, layout, B, H, Sk, D)) != FA_OK) return st;
+  if ((st = make_map(&mv, v, dtype, layout, B, H, Sk, D)) != FA_OK) return st;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* lse_part = reinterpret_cast<float*>(ws + 256);
+  const size_t prow = (size_t)(B * H * n_eff * Sq);
+  float* o_part = reinterpret_cast<float*>(ws + 256 + ((prow * 4 + 15) & ~(size_t)15));
+
+  fa::Params prm{};
+  prm.lse = lse_part;
+  prm.acc = o_part;
+  prm.o = static_cast<uint8_t*>(o);        // not written: every split's result is a partial
+  prm.o_bs = H * n_eff * Sq * D;
+  prm.o_hs = n_eff * Sq * D;
+  prm.o_rs = D;
+  prm.lse_bs = H * n_eff * Sq;
+  prm.lse_hs = n_eff * Sq;
+  prm.B = (int)B;
+  prm.H = (int)H;
+  prm.Sq = (int)Sq;
+  prm.Sk = (int)Sk;
+  prm.nqb = (int)nqb;
+  prm.tk = (int)((split_keys + fa::BN - 1) / fa::BN);
+  prm.bh = (int)(B * H);
+  prm.head0 = 0;
+  prm.group_heads = l2_group_heads(split_keys, D, B * H);
+  prm.total_units = (int)(n_eff * B * H * nqb);
+  prm.causal = 0;
+  prm.bhsd = layout == FA_BHSD ? 1 : 0;
+  prm.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  prm.wait_limit_ns = 1000000000ull;
+  prm.withhold_loads = 0;
+  set_softmax_params(prm, SoftmaxOpts());
+  prm.nseg = 1;                 // the ring-step kind, in its split mode
+  prm.seg_units0 = (int)(B * H * nqb);
+  prm.split_n = (int)n_eff;
+  prm.split_keys = (int)split_keys;
+  st = launch_units(prm, mq, mk, mv, mq, D, dtype, reinterpret_cast<unsigned int*>(ws), dev, sms, stream);
+  if (st != FA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long rows = B * H * Sq;
+  const unsigned grid = (unsigned)((rows + fa::merge::THREADS / 32 - 1) / (fa::merge::THREADS / 32));
+  uint16_t* o16 = static_cast<uint16_t*>(o);
+  const int bhsd = layout == FA_BHSD ? 1 : 0;
+  if (D == 128) {
+    if (dtype == FA_BF16)
+      fa::merge::splitkv_merge_kernel<128, true><<<grid, fa::merge::THREADS, 0, s>>>(o_part, lse_part, o16, lse, rows, (int)H, (int)Sq, (int)n_eff, bhsd);
+    else
+      fa::merge::splitkv_merge_kernel<128, false><<<grid, fa::merge::THREADS, 0, s>>>(o_part, lse_part, o16, lse, rows, (int)H, (int)Sq, (int)n_eff, bhsd);
+  } else {
+    if (dtype == FA_BF16)
+      fa::merge::splitkv_merge_kernel<64, true><<<grid, fa::merge::THREADS, 0, s>>>(o_part, lse_part, o16, lse, rows, (int)H, (int)Sq, (int)n_eff, bhsd);
+    else
+      fa::merge::splitkv_merge_kernel<64, false><<<grid, fa::merge::THREADS, 0, s>>>(o_part, lse_part, o16, lse, rows, (int)H, (int)Sq, (int)n_eff, bhsd);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail((int)e);
+  return FA_OK;
 }
 
 }  // extern "C"

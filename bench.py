@@ -39,6 +39,10 @@ replaced by lookups) and reports each virtual rank's share of the flops over
 its own time; the value projects W GPUs as the whole sequence's flops over
 the slowest virtual rank's time.
 
+--splitkv [N] times the workload (no mask only) through fa_fwd_splitkv, the
+keys split into N ranges (default: enough work units for every SM), next to
+the one-pass kernel on the same inputs.
+
 --proj times attention followed by its output projection (fa_fwd_proj:
 y = o w_o^T with E = H * D output features, w_o seeded N(0, 1/(H D))) on the
 same workload; the value counts both parts' flops, and the attention kernel
@@ -202,6 +206,9 @@ def bench_workload(args):
     if args.bh:
         b, h = (int(x) for x in args.bh.split(","))
         w = w.with_(B=b, H=h, name=f"{w.name}_b{b}_h{h}")
+    if getattr(args, "sqsk", None):
+        sq, sk = (int(x) for x in args.sqsk.split(","))
+        w = w.with_(Sq=sq, Sk=sk, name=f"{w.name}_q{sq}_k{sk}")
     return w
 
 
@@ -625,6 +632,74 @@ def run_ring_emulated(args, w, dev):
     }
 
 
+def run_splitkv(args, rank, world, local_rank):
+    """--splitkv [N]: the workload (no mask) through fa_fwd_splitkv, N key ranges (0: the binding's default
+    for this size), timed next to the one-pass kernel on the same inputs; one JSON line."""
+    import attention_forward_19_b200 as fa
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world != 1:
+        raise SystemExit("--splitkv runs on one GPU")
+    w = bench_workload(args)
+    if w.causal:
+        raise SystemExit("--splitkv applies no mask: pick a workload without causal masking")
+    q, k, v = make_qkv(w, device=dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    n = args.splitkv if args.splitkv > 0 else fa.default_splits(w.B, w.H, w.Sq, w.Sk, sms)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.Sq), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.fa_fwd_splitkv_workspace_size(w.B, w.H, w.Sq, w.D, n), dtype=torch.uint8, device=dev)
+    ws1 = torch.empty(fa.fa_fwd_workspace_size(), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def split():
+        fa.flash_attention_forward_splitkv(q, k, v, layout=w.layout, scale=w.scale, nsplit=n, out=o, lse=lse,
+                                           workspace=ws, stream=stream)
+
+    def one_pass():
+        fa.flash_attention_forward(q, k, v, layout=w.layout, causal=False, scale=w.scale, out=o, lse=lse,
+                                   workspace=ws1, stream=stream)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / args.steps
+
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    clocks = ClockSampler(cvd.split(",")[local_rank].strip() if cvd else str(local_rank))
+    clocks.start()
+    time.sleep(0.3)
+    ms_one = timed(one_pass)
+    ms = timed(split)
+    clk = clocks.stop()
+    fa.check_device_status(stream)
+    flops = w.flops()
+    value = flops / (ms * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    cfg = workload_config(w, 1)
+    cfg.update({"global_batch": w.B, "parallelism": f"split-KV: {n} key ranges, partials merged by a second kernel"})
+    return {
+        "metric": "attn fwd TFLOP/s, split-KV (fa_fwd_splitkv: the keys split across CTAs)", "value": value,
+        "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": cfg,
+        "one_pass_ms_per_step": ms_one, "one_pass_value": flops / (ms_one * 1e-3) / 1e12,
+        "roofline": {"bound": "tensor", "achieved": value, "peak": peak, "unit": UNIT, "frac": value / peak,
+                     "traffic": None, "peak_source": f"{peak_kind} bf16 burst (MEASURED_PEAKS.json bf16_tflops)"},
+        "gpu_launches": 2 * args.steps,
+        "gpu_launches_note": "per step: the ring-step kernel in its split mode and the merge kernel",
+        "clocks": clk,
+    }
+
+
 def run_proj(args, rank, world, local_rank):
     """Times attention + output projection (fa_fwd_proj) and each kernel alone (one JSON line)."""
     import attention_forward_19_b200 as fa
@@ -755,10 +830,14 @@ def main():
     ap.add_argument("--workload", choices=list(WORKLOADS), default=None,
                     help=f"default {BENCH_WORKLOAD} ({RING_WORKLOAD} with --ring)")
     ap.add_argument("--bh", default=None, help="override B,H of the workload (profiling runs)")
+    ap.add_argument("--sqsk", default=None, help="override Sq,Sk of the workload (profiling and split-KV runs)")
     ap.add_argument("--backward", action="store_true", help="time the backward pass instead (its own JSON line)")
     ap.add_argument("--atomic", action="store_true", help="with --backward: the non-deterministic variant")
     ap.add_argument("--ring", action="store_true", help="time ring attention of one sequence over the ranks")
     ap.add_argument("--proj", action="store_true", help="time attention + output projection (fa_fwd_proj)")
+    ap.add_argument("--splitkv", type=int, default=-1, nargs="?", const=0,
+                    help="time the workload (no mask) through fa_fwd_splitkv with this many key ranges (0 or no "
+                         "value: the default for its size) next to the one-pass kernel")
     ap.add_argument("--emulate-ranks", type=int, default=0,
                     help="with --ring on one GPU: time the schedule of this many virtual ranks")
     ap.add_argument("--strong", action="store_true",
@@ -784,7 +863,7 @@ def main():
                                                  device_id=torch.device("cuda", local_rank))
         try:
             run = (run_ring if args.ring else run_proj if args.proj else run_backward if args.backward
-                   else run_native)
+                   else run_splitkv if args.splitkv >= 0 else run_native)
             line = run(args, rank, world, local_rank)
         finally:
             if world > 1:

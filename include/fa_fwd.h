@@ -41,7 +41,7 @@
  * the end; LSE is fp32.
  *
  * Besides the forward pass (fa_fwd, fa_fwd_ws, fa_fwd_opts, fa_fwd_heads,
- * fa_fwd_noalloc, fa_fwd_varlen) the library exports its backward pass
+ * fa_fwd_noalloc, fa_fwd_varlen, fa_fwd_splitkv) the library exports its backward pass
  * (fa_bwd, fa_bwd_atomic), the merge of
  * partial results that ring attention over several GPUs is built from
  * (fa_lse_merge), one ring step with that merge fused into the attention
@@ -461,6 +461,35 @@ fa_status fa_fwd_ring_step(const void *q, const void *k, const void *v, void *o,
                            int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D, int64_t rows,
                            const fa_ring_segment *segs, int nseg, fa_layout layout, float scale,
                            fa_dtype dtype, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * fa_fwd_splitkv -- the forward pass without a mask for problems with few
+ * work units (few heads and query rows: a short prompt, or decoding against a
+ * long key sequence), with the keys split across CTAs as well.  The key range
+ * is cut into up to nsplit ranges of whole 128-key tiles; every (query rows,
+ * key range) pair is a work unit of the ring-step kernel, which writes the
+ * range's result normalised over its own keys (fp32 O and LSE, in the
+ * workspace); a second kernel merges a row's partial results by the update
+ * of fa_lse_merge taken over all of them at once (page "FlashAttention: long-
+ * text inference without running out of memory" (ai6s.net/6a0d42d8), section
+ * on tiling and online normalisation, applied to whole key ranges):
+ *     LSE = log(sum_s exp(LSE_s)),  O = sum_s exp(LSE_s - LSE) O_s
+ * and writes O (rounded to nearest in dtype) and LSE as fa_fwd does.  The
+ * result equals fa_fwd's within rounding (the partial results are fp32), not
+ * bit for bit.
+ *
+ * Arguments as for fa_fwd with causal = 0 (no mask is applied), plus
+ * nsplit     1..64 requested key ranges (fewer when Sk has fewer 128-key tiles)
+ * workspace  fa_fwd_splitkv_workspace_size(B, H, Sq, D, nsplit) bytes of
+ *            caller-owned device memory, 256-byte aligned, not overlapping
+ *            any tensor (FA_ERR_ALIAS); overwritten by the call
+ * Errors as for fa_fwd_ws; FA_ERR_INVALID_ARG for nsplit outside 1..64 or a
+ * missing or short workspace.  Asynchronous on `stream`.
+ */
+size_t fa_fwd_splitkv_workspace_size(int64_t B, int64_t H, int64_t Sq, int64_t D, int nsplit);
+fa_status fa_fwd_splitkv(const void *q, const void *k, const void *v, void *o, float *lse, int64_t B, int64_t H,
+                         int64_t Sq, int64_t Sk, int64_t D, fa_layout layout, float scale, fa_dtype dtype,
+                         int nsplit, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * fa_out_proj -- the attention output projection Y = O W^T (page "catlass

@@ -414,3 +414,51 @@ def test_bwd_atomic_workspace_and_validation(lib):
     # D = 64: its own accumulator size; a D = 128 workspace is large enough, a deterministic one is not
     assert fa.fa_bwd_atomic_workspace_size(1, 2, 64, 64) == 2 * 128 * (2 + 64) * 4
     assert call(D=64, ws_bytes=fa.fa_bwd_workspace_size(1, 2, 64)) == fa.FA_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------- split-KV (fa_fwd_splitkv)
+
+SKW = 0x70000000     # a 256-byte aligned fake workspace, far from the fake tensors
+
+
+def call_split(ws=SKW, ws_bytes=None, nsplit=4, **kw):
+    a = dict(GOOD)
+    a.update(kw)
+    if ws_bytes is None:
+        ws_bytes = max(256, fa.fa_fwd_splitkv_workspace_size(a["B"], a["H"], max(a["Sq"], 0), a["D"], nsplit))
+    return fa.fa_fwd_splitkv(Q, K, V, O, L, a["B"], a["H"], a["Sq"], a["Sk"], a["D"], a["layout"], a["scale"],
+                             a["dtype"], nsplit, ws, ws_bytes, None)
+
+
+def test_splitkv_workspace_size(lib):
+    B, H, Sq, D = 2, 3, 300, 128
+    for n in (1, 4, 64):
+        rows = B * H * n * Sq
+        assert fa.fa_fwd_splitkv_workspace_size(B, H, Sq, D, n) == 256 + (rows * 4 + 15) // 16 * 16 + rows * D * 4
+    assert fa.fa_fwd_splitkv_workspace_size(B, H, Sq, 64, 8) < fa.fa_fwd_splitkv_workspace_size(B, H, Sq, 128, 8)
+    for bad in (dict(nsplit=0), dict(nsplit=65), dict(D=96), dict(B=0), dict(H=-1), dict(Sq=-1)):
+        a = dict(B=B, H=H, Sq=Sq, D=D, nsplit=4)
+        a.update(bad)
+        assert fa.fa_fwd_splitkv_workspace_size(a["B"], a["H"], a["Sq"], a["D"], a["nsplit"]) == 0, bad
+
+
+def test_splitkv_host_validation(lib):
+    for kw in (dict(B=0), dict(layout=3), dict(dtype=5), dict(scale=float("nan")), dict(nsplit=0),
+               dict(nsplit=65), dict(ws=0), dict(ws_bytes=255)):
+        assert call_split(**kw) == fa.FA_ERR_INVALID_ARG, kw
+    # the workspace must hold nsplit splits' partials: one byte short is refused
+    need = fa.fa_fwd_splitkv_workspace_size(GOOD["B"], GOOD["H"], GOOD["Sq"], GOOD["D"], 4)
+    assert call_split(ws_bytes=need - 1) == fa.FA_ERR_INVALID_ARG
+    assert call_split(ws=SKW + 16) == fa.FA_ERR_MISALIGNED
+    assert call_split(ws=Q) == fa.FA_ERR_ALIAS
+    assert call_split(D=96) == fa.FA_ERR_UNSUPPORTED
+    assert call_split(Sq=0) == fa.FA_OK
+
+
+def test_default_splits():
+    assert fa.default_splits(1, 2, 512, 512) == 1            # 4 key tiles: too short to split
+    assert fa.default_splits(1, 2, 512, 8192) == 8           # 64 tiles, 8 per range
+    assert fa.default_splits(1, 8, 128, 65536) == 18         # 8 units: 148 // 8
+    assert fa.default_splits(4, 8, 512, 32768) == 2          # 64 units
+    assert fa.default_splits(2, 40, 8192, 8192) == 1         # already thousands of units
+    assert fa.default_splits(1, 1, 1, 1000000) == 64         # capped at 64
