@@ -128,33 +128,47 @@ __global__ void __launch_bounds__(THREADS) splitkv_merge_kernel(const float* __r
   const long long bh = row / S;
   const int r = (int)(row - bh * S);
   const size_t base = (size_t)bh * nsplit * S + r;
-  float m = -INFINITY;
-  for (int s = lane; s < nsplit; s += 32) m = fmaxf(m, lse_part[base + (size_t)s * S]);
+  // lane l holds the LSEs of splits l and l + 32 (nsplit <= 64) and their weights
+  const float l0 = lane < nsplit ? lse_part[base + (size_t)lane * S] : -INFINITY;
+  const float l1 = lane + 32 < nsplit ? lse_part[base + (size_t)(lane + 32) * S] : -INFINITY;
+  float m = fmaxf(l0, l1);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  const float e0 = (m > -INFINITY && l0 > -INFINITY) ? ex2((l0 - m) * LOG2E) : 0.f;
+  const float e1 = (m > -INFINITY && l1 > -INFINITY) ? ex2((l1 - m) * LOG2E) : 0.f;
+  float wsum = e0 + e1;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
   float acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-  float wsum = 0.f;
-  if (m > -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float ls = lse_part[base + (size_t)s * S];
-      if (!(ls > -INFINITY)) continue;
-      const float w = ex2((ls - m) * LOG2E);
-      wsum += w;
-      const float* src = o_part + (base + (size_t)s * S) * D + lane * PER;
-      if constexpr (PER == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(src);
-        acc[0] += w * x.x;
-        acc[1] += w * x.y;
-        acc[2] += w * x.z;
-        acc[3] += w * x.w;
+  // four splits' rows in flight at a time (a split of weight 0 is not read)
+  for (int s0 = 0; s0 < nsplit; s0 += 4) {
+    float w[4];
+    float x[4][PER];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int sp = s0 + u;
+      const float e = __shfl_sync(0xffffffffu, sp < 32 ? e0 : e1, sp & 31);
+      w[u] = sp < nsplit ? e : 0.f;
+      const float* src = o_part + (base + (size_t)sp * S) * D + lane * PER;
+      if (w[u] != 0.f) {
+        if constexpr (PER == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(src);
+          x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(src);
+          x[u][0] = v.x; x[u][1] = v.y;
+        }
       } else {
-        const float2 x = *reinterpret_cast<const float2*>(src);
-        acc[0] += w * x.x;
-        acc[1] += w * x.y;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) x[u][i] = 0.f;
       }
     }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] += w[u] * x[u][i];
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   const long long b = bh / H, h = bh - b * H;
