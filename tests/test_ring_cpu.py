@@ -70,17 +70,24 @@ def test_every_visible_key_is_used_exactly_once(world, causal):
     assert np.array_equal(count, mask)
 
 
+def reversed_zigzag(rank, world):
+    """The zigzag pair in the other order: a rank's held chunks are then not in ascending order, so a
+    step can need a segment that starts at the second held chunk, or two segments for one query chunk."""
+    return (2 * world - 1 - rank, rank)
+
+
 @pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
 @pytest.mark.parametrize("causal", [False, True])
-def test_step_segments_cover_every_visible_key_exactly_once(world, causal):
+@pytest.mark.parametrize("ids", [ring.zigzag_chunk_ids, reversed_zigzag], ids=["zigzag", "reversed"])
+def test_step_segments_cover_every_visible_key_exactly_once(world, causal, ids):
     # the fa_fwd_ring_step segments of every rank and step, expanded to (global row, global key) pairs
     Sc = 3
     S = 2 * world * Sc
     count = np.zeros((S, S), dtype=int)
     for r in range(world):
-        mine = ring.zigzag_chunk_ids(r, world)
-        for t, segs in enumerate(ring.step_plan(r, world, causal)):
-            held = ring.zigzag_chunk_ids(ring.ring_source(r, world, t), world)
+        mine = ids(r, world)
+        for t, segs in enumerate(ring.step_plan(r, world, causal, ids)):
+            held = ids(ring.ring_source(r, world, t), world)
             for (row0, key0, keys, off, _, _) in ring.fa_segments(segs, Sc):
                 for rr in range(Sc):
                     grow = mine[(row0 + rr) // Sc] * Sc + (row0 + rr) % Sc
@@ -110,6 +117,16 @@ def test_step_plan_first_and_last_and_one_launch_per_step(world, causal):
     # with causal zigzag chunks every step has work on every rank
     if causal:
         assert all(ring.step_plan(r, world, True)[t] for r in range(world) for t in range(world))
+
+
+def test_reversed_pairs_need_later_key_chunks_and_two_launches():
+    plan = ring.step_plan(0, 2, True, reversed_zigzag)
+    # step 0: query chunk 0 (global 3) sees held chunk 0 (global 3, the diagonal) and then chunk 1 (global 0,
+    # fully visible): two segments for one query chunk, so two launches; query chunk 1 (global 0) sees
+    # only held chunk 1 (key0 = Sc), its diagonal
+    assert plan[0] == [(0, 0, 1, True, True, False), (0, 1, 2, False, False, False), (1, 1, 2, True, True, True)]
+    assert [len(b) for b in ring.launch_batches(plan[0])] == [2, 1]
+    assert ring.fa_segments([plan[0][2]], 5) == [(5, 5, 5, 0, 1, 1)]
 
 
 def test_launch_batches_split_repeated_query_chunks():
@@ -145,12 +162,13 @@ def test_shard_unshard_round_trip(layout):
 @pytest.mark.parametrize("world", [1, 2, 3, 4])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("layout", ["BSND", "BHSD"])
-def test_emulated_ring_with_oracle_steps_matches_whole_attention(world, causal, layout):
+@pytest.mark.parametrize("ids", [ring.zigzag_chunk_ids, reversed_zigzag], ids=["zigzag", "reversed"])
+def test_emulated_ring_with_oracle_steps_matches_whole_attention(world, causal, layout, ids):
     q, k, v = _qkv(layout, S=2 * world * 6)
     scale = 0.3
     ops = OracleOps(layout, scale)
     o, l = ring.ring_attention_emulated(q, k, v, world, causal=causal, scale=scale, layout=layout,
-                                        ops=ring.BlockwiseStep(ops))
+                                        ops=ring.BlockwiseStep(ops), chunk_ids_of=ids)
     o_ref, l_ref = _oracle_whole(q, k, v, layout, causal, scale)
     assert float((o - o_ref).abs().max()) < 1e-12
     assert float((l - l_ref).abs().max()) < 1e-12

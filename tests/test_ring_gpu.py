@@ -210,6 +210,24 @@ def test_emulated_ring_matches_oracle(orc, case):
     assert err_o <= O_TOL[dtype] and err_l <= LSE_TOL
 
 
+@pytest.mark.parametrize("world,layout", [(2, "BSND"), (3, "BHSD")])
+def test_emulated_ring_with_reversed_pairs_matches_oracle(orc, world, layout):
+    # held chunks in descending order: segments that start at the second held chunk, and steps that need
+    # two fa_fwd_ring_step launches (two segments of one query chunk)
+    _need_gpu()
+    ids = lambda r, w: (2 * w - 1 - r, r)
+    dtype, S, D = torch.bfloat16, 2 * world * 150, 128
+    q, k, v = _qkv(layout, dtype, 1, 2, S, D, seed=S + 7)
+    o, lse = ring.ring_attention_emulated(q.cuda(), k.cuda(), v.cuda(), world, causal=True, layout=layout,
+                                          chunk_ids_of=ids)
+    fa.check_device_status()
+    o_ref, l_ref = orc.fwd(q, k, v, layout=layout, causal=True, scale=1.0 / math.sqrt(D))
+    err_o = float(np.max(np.abs(_head_major(o, layout) - o_ref)))
+    err_l = float(np.max(np.abs(lse.double().cpu().numpy() - l_ref)))
+    print(f"PARITY ring reversed w{world} {layout}: max|dO| {err_o:.3e} max|dLSE| {err_l:.3e}")
+    assert err_o <= O_TOL[dtype] and err_l <= LSE_TOL
+
+
 def test_ring_forward_without_process_group_is_plain_attention(orc):
     _need_gpu()
     import torch.distributed as dist
