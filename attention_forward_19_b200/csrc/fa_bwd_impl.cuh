@@ -340,6 +340,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ---- phase A: P^T = 2^(s c - lse2) from S^T, packed to the input dtype
       // (phase B takes P from these packed words: it is the P the tile
       // products use, and half the registers of an fp32 copy)
+      // the group's lse2 values are read before the wait: their shared-memory
+      // latency then overlaps the wait instead of following it
+      float4 lv4[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) lv4[i] = *reinterpret_cast<const float4*>(vl + grp * 64 + 4 * i);
       ok = wait_bar(bar(C::S_FULL), n & 1u, abort_flag, limit);
       if (!ok) break;
       tc_fence_after();
@@ -354,7 +359,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int qa = col + 2 * e;
-          const float4 l4 = *reinterpret_cast<const float4*>(vl + (qa & ~3));
+          const float4 l4 = lv4[ch * 8 + (e >> 1)];
           const float la = (qa & 2) ? l4.z : l4.x, lb = (qa & 2) ? l4.w : l4.y;
           float pa = ex2(fmaf(__uint_as_float(sv[2 * e]), c, -la));
           float pb = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, -lb));
@@ -372,6 +377,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       mbar_arrive(bar(C::W_A));
       // ---- phase B: dS^T = P^T (dP^T - D)
+      float4 dv4[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) dv4[i] = *reinterpret_cast<const float4*>(vd + grp * 64 + 4 * i);
       ok = wait_bar(bar(C::DP_FULL), n & 1u, abort_flag, limit);
       if (!ok) break;
       tc_fence_after();
@@ -386,7 +394,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int qa = col + 2 * e;
-          const float4 d4 = *reinterpret_cast<const float4*>(vd + (qa & ~3));
+          const float4 d4 = dv4[ch * 8 + (e >> 1)];
           const float da = (qa & 2) ? d4.z : d4.x, db = (qa & 2) ? d4.w : d4.y;
           const float2 pp = unpack2(pk[ch * 16 + e], BF16);
           pg[ch * 16 + e] = pack2<BF16>(pp.x * (__uint_as_float(dp[2 * e]) - da), pp.y * (__uint_as_float(dp[2 * e + 1]) - db));
